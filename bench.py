@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A4 NVFP4 linear hot path on B200.
+
+One step = one pass of the whole hot path over one batch: tensor amax, fused
+smooth/quantise/pack + low-rank down-projection, and the block-scaled FP4 GEMM
+with the low-rank up-projection, bias and bf16 cast, on the FLUX-1024px QKV
+projection (M = 4608 tokens = 4096 image + 512 text, K = 3072, N = 9216,
+rank 32, bf16 bias).  Inputs are synthetic (seeded), shaped like that workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  Under torchrun (N > 1) every rank runs an independent
+replica on its own GPU (the path has no cross-GPU exchange); rank 0 prints.
+``--impl reference`` times the plain CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = {"workload": "FLUX-1024px QKV projection", "M": 4608, "K": 3072, "N": 9216, "r": 32,
+            "bias": True, "activation": "N(0,1) with 1% Student-t(2)x50 channels", "weight": "N(0,0.02)"}
+METRIC = "W4A4 linear TFLOPS (act-quant+FP4 GEMM+low-rank)"
+L2_SETS = 3          # rotating buffer sets, each ~140 MB, so every step starts L2-cold
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_per_step(M, K, N, r):
+    return 2.0 * M * N * K + 2.0 * M * r * (K + N)
+
+
+def gemm_flops(M, K, N, r):
+    return 2.0 * M * N * K + 2.0 * M * N * (2 * r)  # main GEMM + the hi/lo low-rank pass
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def ncu_traffic(kernel_src: str, summary: str):
+    """DRAM bytes per launch from the committed ncu summary, if that summary
+    was taken on the current kernel source (hash match); else None."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", text)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()
+    if not cur.startswith(h.group(1)):
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return []
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            rows.append(parts)
+        return rows
+
+    @staticmethod
+    def summarise(rows, sm_floor=300.0):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = []
+        reasons = set()
+        max_mhz = None
+        for r in rows:
+            try:
+                mhz = float(r[1])
+                max_mhz = float(r[2])
+            except ValueError:
+                continue
+            if mhz < sm_floor:
+                continue
+            sm.append(mhz)
+            for n, v in zip(names, r[4:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max_mhz,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def build_inputs(torch, w4, prep, dev):
+    from synth import config_cases, bf16_bits
+    case = config_cases(2)[0]
+    M, K, N, r = case.M, case.K, case.N, case.r
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(bf16_bits(a).view(np.int16))).to(dev).view(torch.bfloat16)
+
+    W = dev_bf16(case.w)
+    Xc = dev_bf16(case.x_cal)
+    bias = dev_bf16(case.bias)
+    packed = prep.svdquant_prepare(W, Xc, r=r, bias=bias)
+    del W, Xc
+    x_host = np.ascontiguousarray(bf16_bits(case.x).view(np.int16))
+    sets = []
+    for i in range(L2_SETS):
+        X = torch.from_numpy(x_host).to(dev).view(torch.bfloat16)
+        w = w4.PackedWeight(packed.Wq.clone(), packed.Wsf.clone(), packed.t_w.clone(), N, K,
+                            packed.inv_s.clone(), packed.L1t.clone(), packed.L2t.clone(), packed.bias.clone())
+        qa = w4.QuantizedActivation(
+            torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+            torch.empty(w4.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev),
+            torch.empty(1, dtype=torch.float32, device=dev),
+            torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev), M, K, r)
+        ws = torch.empty(w4.nvfp4_quant_workspace_bytes(M, K, r), dtype=torch.uint8, device=dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        sets.append((X, w, qa, ws, Y))
+    return case, x_host, sets
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("gloo", timeout=__import__("datetime").timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import bit_diffusion_transformer_nvfp4_b200 as w4
+    from bit_diffusion_transformer_nvfp4_b200 import prep
+    w4.lib()
+
+    case, x_host, sets = build_inputs(torch, w4, prep, dev)
+    M, K, N, r = case.M, case.K, case.N, case.r
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev_mid=None):
+        X, w, qa, ws, Y = sets[i % L2_SETS]
+        w4.nvfp4_quantize_act(X, M, K, K, w.inv_s, w.L1t, r, w.t_w, qa.Xq, qa.Xsf, qa.t_x, qa.U, ws, stream)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        w4.w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, w.Wq, w.Wsf, w.t_w, w.L2t, r, w.bias, 0, Y, N, stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step(i, evs[i][1])
+        evs[i][2].record(stream)
+    barrier()
+    t_wall1 = time.time()
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    quant_ms = [e[0].elapsed_time(e[1]) for e in evs]
+
+    # end to end through the public API with host buffers: pinned X in,
+    # linear on the device, pinned Y out, every step
+    import torch as _t
+    xh = _t.from_numpy(x_host).view(_t.bfloat16).pin_memory()
+    yh = _t.empty(M, N, dtype=_t.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    X0, w0, qa0, ws0, Y0 = sets[0]
+    lin_ws = torch.empty(w4.w4a4_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    for i in range(2):
+        X0.copy_(xh, non_blocking=True)
+        w4.w4a4_linear(X0, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y0, lin_ws, stream)
+        yh.copy_(Y0, non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        X0.copy_(xh, non_blocking=True)
+        w4.w4a4_linear(X0, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y0, lin_ws, stream)
+        yh.copy_(Y0, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    clock_rows = sampler.stop()
+    status = w4.w4a4_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {w4.w4a4_status_string(status)}")
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    fl = flops_per_step(M, K, N, r)
+    ms_per_step = total_ms / args.steps
+    value = world * fl * args.steps / (total_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_avg_ms = statistics.mean(gemm_ms)
+    g_fl = gemm_flops(M, K, N, r)
+    achieved = g_fl / (gemm_avg_ms * 1e-3) / 1e12
+    traffic = ncu_traffic("bit_diffusion_transformer_nvfp4_b200/csrc/gemm.cuh", "gemm_flux1024_qkv_ncu.md")
+    clocks = ClockSampler.summarise(clock_rows)
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       l2=f"{L2_SETS} rotating input/weight/output sets of ~140 MB each (> 126 MB L2)"),
+        "pct_fp4_peak": round(100.0 * value / (world * fp4_peak), 2),
+        "fp4_peak_tflops": round(fp4_peak, 1),
+        "fp4_peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOPS x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
+        "roofline": {"kernel": "gemm_kernel (block-scaled FP4 + low-rank + bias epilogue)", "bound": "tensor",
+                     "achieved": round(achieved, 2), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
+                     "peak_kind": f"{peak_kind} (bf16 burst x4)", "launch_ms": round(gemm_avg_ms, 5),
+                     "algorithmic_flops_per_launch": g_fl},
+        "kernels_ms": {"amax+quant": round(statistics.mean(quant_ms), 5), "gemm": round(gemm_avg_ms, 5)},
+        "e2e": {"value": round(world * fl / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2),
+                "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "wall_s_timed": round(t_wall1 - t_wall0, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(case, sample_rows=args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- oracle arms
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_prepared(case):
+    from oracle import nvfp4, prep
+    p = prep.svdquant_prepare(case.w, case.x_cal, case.r, case.alpha)
+    wq, wsf, tw, _ = nvfp4.quantize_activation(p["R"], None)
+    return p, wq, wsf, tw
+
+
+def cpu_baseline(case, sample_rows=512, prepared=None):
+    """The oracle as it stands on a bounded sample: the whole activation is
+    quantised (the tensor scale needs every row) and Y is formed for
+    ``sample_rows`` rows; throughput counts the sampled rows' FLOPs."""
+    from oracle import linear as olinear
+    p, wq, wsf, tw = prepared or oracle_prepared(case)
+    rows = np.sort(np.random.Generator(np.random.PCG64(7)).choice(case.M, sample_rows, replace=False))
+    t0 = time.perf_counter()
+    olinear.w4a4_linear(case.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"], case.bias, rows=rows)
+    dt = time.perf_counter() - t0
+    fl = flops_per_step(sample_rows, case.K, case.N, case.r)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"whole-tensor activation quantisation + Y for {sample_rows} of {case.M} rows "
+                      f"(numpy fp32 quantiser, fp64 matmul), {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from synth import config_cases
+    case = config_cases(2)[0]
+    prepared = oracle_prepared(case)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        cpu_baseline(case, rows, prepared)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_baseline(case, rows, prepared)
+    dt = time.perf_counter() - t0
+    fl = flops_per_step(rows, case.K, case.N, case.r)
+    value = fl * args.steps / dt / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": 0,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": dict(WORKLOAD, parallelism="host CPU"),
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cpu_threads(), "kind": "oracle",
+                            "sample": f"per step: whole-tensor activation quantisation + Y for {rows} of {case.M} rows"},
+           "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

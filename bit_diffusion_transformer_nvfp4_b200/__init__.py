@@ -1,0 +1,210 @@
+"""B200 (sm_100a) W4A4 NVFP4 linear layer: Python binding of ``libw4a4.so``.
+
+Every function here marshals arguments (tensor pointers, sizes, the current
+CUDA stream) into the C ABI declared in ``include/w4a4.h`` and raises on a
+non-zero status.  All arithmetic runs in the CUDA kernels of the shared
+library; there is no CPU or PyTorch fallback: if the library is missing the
+import of any wrapper raises.
+
+PyTorch is used only for device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "lib", "W4A4Error", "nvfp4_sf_bytes", "nvfp4_quant_workspace_bytes", "w4a4_workspace_bytes",
+    "nvfp4_quantize_act", "nvfp4_pack_weight", "w4a4_gemm", "w4a4_linear", "w4a4_device_status",
+    "w4a4_status_string", "EPI_NONE", "EPI_GELU_TANH", "SRC_BF16", "SRC_F32",
+    "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libw4a4.so")
+
+EPI_NONE, EPI_GELU_TANH = 0, 1
+SRC_BF16, SRC_F32 = 0, 1
+
+_c = ctypes
+_P = _c.c_void_p
+_I64 = _c.c_int64
+_SIG = {
+    "nvfp4_sf_bytes": (_c.c_size_t, [_I64, _I64]),
+    "nvfp4_quant_workspace_bytes": (_c.c_size_t, [_I64, _I64, _c.c_int]),
+    "w4a4_workspace_bytes": (_c.c_size_t, [_I64, _I64, _I64, _c.c_int]),
+    "nvfp4_quantize_act": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P, _P,
+                                      _c.c_size_t, _P]),
+    "nvfp4_pack_weight": (_c.c_int, [_P, _c.c_int, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_size_t, _P]),
+    "w4a4_gemm": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _c.c_int,
+                             _P, _I64, _P]),
+    "w4a4_linear": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _c.c_int, _P, _c.c_int, _P,
+                               _P, _c.c_size_t, _P]),
+    "w4a4_device_status": (_c.c_int, [_c.POINTER(_c.c_int), _c.c_int]),
+    "w4a4_status_string": (_c.c_char_p, [_c.c_int]),
+}
+
+_lib = None
+
+
+class W4A4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed with status {status}: {w4a4_status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (built by ``build.py``); raises if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m bit_diffusion_transformer_nvfp4_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIG.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise W4A4Error(fn, st)
+
+
+# ------------------------------------------------------------------ raw ABI
+
+def nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return lib().nvfp4_sf_bytes(rows, K)
+
+
+def nvfp4_quant_workspace_bytes(M: int, K: int, r: int) -> int:
+    return lib().nvfp4_quant_workspace_bytes(M, K, r)
+
+
+def w4a4_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return lib().w4a4_workspace_bytes(M, N, K, r)
+
+
+def w4a4_status_string(status: int) -> str:
+    return lib().w4a4_status_string(status).decode()
+
+
+def nvfp4_quantize_act(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, workspace, stream=None):
+    _check("nvfp4_quantize_act", lib().nvfp4_quantize_act(
+        _ptr(X), M, K, ldx, _ptr(inv_s), _ptr(L1t), r, _ptr(t_w), _ptr(Xq), _ptr(Xsf), _ptr(t_x),
+        _ptr(U), _ptr(workspace), workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream(stream)))
+
+
+def nvfp4_pack_weight(R, src_dtype, N, K, ldr, Wq, Wsf, t_w, workspace, stream=None):
+    _check("nvfp4_pack_weight", lib().nvfp4_pack_weight(
+        _ptr(R), src_dtype, N, K, ldr, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(workspace),
+        workspace.numel() * workspace.element_size() if workspace is not None else 0, _stream(stream)))
+
+
+def w4a4_gemm(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, stream=None):
+    _check("w4a4_gemm", lib().w4a4_gemm(
+        _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
+        _ptr(bias), epilogue, _ptr(Y), ldy, _stream(stream)))
+
+
+def w4a4_linear(X, M, N, K, Wq, Wsf, t_w, inv_s, L1t, L2t, r, bias, epilogue, Y, workspace, stream=None):
+    _check("w4a4_linear", lib().w4a4_linear(
+        _ptr(X), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(inv_s), _ptr(L1t), _ptr(L2t), r, _ptr(bias),
+        epilogue, _ptr(Y), _ptr(workspace),
+        workspace.numel() * workspace.element_size() if workspace is not None else 0, _stream(stream)))
+
+
+def w4a4_device_status(reset: bool = False) -> int:
+    v = ctypes.c_int(0)
+    _check("w4a4_device_status", lib().w4a4_device_status(ctypes.byref(v), 1 if reset else 0))
+    return v.value
+
+
+# ------------------------------------------------------------------ tensor-level helpers
+# These allocate outputs with torch (device memory is the caller's business in
+# the C ABI) and call the raw wrappers above.
+
+def _u8(n, device):
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+class QuantizedActivation:
+    """Outputs of nvfp4_quantize_act: codes, SF atoms, tensor scale, low-rank U."""
+
+    def __init__(self, Xq, Xsf, t_x, U, M, K, r):
+        self.Xq, self.Xsf, self.t_x, self.U = Xq, Xsf, t_x, U
+        self.M, self.K, self.r = M, K, r
+
+
+class PackedWeight:
+    """A prepared W4A4 linear: NVFP4 residual weight plus its side inputs."""
+
+    def __init__(self, Wq, Wsf, t_w, N, K, inv_s=None, L1t=None, L2t=None, bias=None):
+        self.Wq, self.Wsf, self.t_w = Wq, Wsf, t_w
+        self.N, self.K = N, K
+        self.inv_s, self.L1t, self.L2t, self.bias = inv_s, L1t, L2t, bias
+        self.r = 0 if L1t is None else int(L1t.shape[0])
+
+
+def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None) -> QuantizedActivation:
+    M, K = X.shape
+    r = 0 if L1t is None else int(L1t.shape[0])
+    dev = X.device
+    Xq = _u8(M * K // 2, dev).view(M, K // 2)
+    Xsf = _u8(nvfp4_sf_bytes(M, K), dev)
+    t_x = torch.empty(1, dtype=torch.float32, device=dev)
+    U = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev) if r else None
+    ws = _u8(max(16, nvfp4_quant_workspace_bytes(M, K, r)), dev)
+    nvfp4_quantize_act(X, M, K, X.stride(0), inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, ws, stream)
+    return QuantizedActivation(Xq, Xsf, t_x, U, M, K, r)
+
+
+def pack_weight(R: torch.Tensor, inv_s=None, L1t=None, L2t=None, bias=None, stream=None) -> PackedWeight:
+    N, K = R.shape
+    dev = R.device
+    src = SRC_F32 if R.dtype == torch.float32 else SRC_BF16
+    Wq = _u8(N * K // 2, dev).view(N, K // 2)
+    Wsf = _u8(nvfp4_sf_bytes(N, K), dev)
+    t_w = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = _u8(max(16, nvfp4_quant_workspace_bytes(N, K, 0)), dev)
+    nvfp4_pack_weight(R, src, N, K, R.stride(0), Wq, Wsf, t_w, ws, stream)
+    return PackedWeight(Wq, Wsf, t_w, N, K, inv_s, L1t, L2t, bias)
+
+
+def gemm(qa: QuantizedActivation, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, stream=None):
+    if Y is None:
+        Y = torch.empty(qa.M, w.N, dtype=torch.bfloat16, device=qa.Xq.device)
+    w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias,
+              epilogue, Y, Y.stride(0), stream)
+    return Y
+
+
+def linear(X: torch.Tensor, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, workspace=None, stream=None):
+    M, K = X.shape
+    if Y is None:
+        Y = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = _u8(max(16, w4a4_workspace_bytes(M, w.N, K, w.r)), X.device)
+    w4a4_linear(X, M, w.N, K, w.Wq, w.Wsf, w.t_w, w.inv_s, w.L1t, w.L2t, w.r, w.bias, epilogue, Y,
+                workspace, stream)
+    return Y

@@ -1,0 +1,386 @@
+// w4a4_api.cu -- the extern "C" entry points declared in include/w4a4.h.
+//
+// Host code only validates arguments, encodes TMA tensor maps, sizes grids
+// and enqueues the kernels of quant.cuh / gemm.cuh on the caller's stream.
+// It never allocates device memory and never synchronises (except
+// w4a4_device_status, which documents that it does).
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/w4a4.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace w4a4 {
+
+// Sticky device status word (W4A4_OK or a device-side error code).
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool ok = false;
+  int num_sms = 0;
+  int* status_ptr = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Per-device set-up: architecture check, SM count, kernel attributes, the
+// device address of the status word.  Returns W4A4_OK or an error.
+int device_setup(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_ARCH; }
+  if (dev < 0 || dev >= kMaxDevices) return W4A4_ERR_ARCH;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.ready) { *out = &d; return d.ok ? W4A4_OK : W4A4_ERR_ARCH; }
+  d.ready = true;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+    cudaGetLastError();
+    return W4A4_ERR_ARCH;
+  }
+  cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status_ptr), g_status) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+      cudaGetLastError();
+      return W4A4_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  bool attr_ok = true;
+  attr_ok &= cudaFuncSetAttribute(quant_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  QuantTile<__nv_bfloat16>::kSmem) == cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(quant_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  QuantTile<float>::kSmem) == cudaSuccess;
+  using G256 = GemmCfg<256, 4>;
+  using G192 = GemmCfg<192, 4>;
+  attr_ok &= cudaFuncSetAttribute(gemm_kernel<G256>, cudaFuncAttributeMaxDynamicSharedMemorySize, G256::SMEM) ==
+             cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(gemm_kernel<G192>, cudaFuncAttributeMaxDynamicSharedMemorySize, G192::SMEM) ==
+             cudaSuccess;
+  if (!attr_ok) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+  d.ok = true;
+  *out = &d;
+  return W4A4_OK;
+}
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scale atoms viewed as u32 [row_blocks][K/64][128]; box (128, 4, rb_box).
+bool encode_sf(CUtensorMap* m, const void* ptr, int64_t rows, int64_t K, uint32_t rb_box) {
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(K / 64), static_cast<cuuint64_t>(ceil_div(rows, 128))};
+  const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(K / 64) * 512};
+  const cuuint32_t box[3] = {128, 4, rb_box};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct QuantPlan {
+  int64_t row_blocks = 0;
+  int chunks = 0, splits = 0, chunks_per_split = 0;
+  size_t off_partials = 0, off_tickets = 0, off_upart = 0, bytes = 0;
+};
+
+QuantPlan quant_plan(int64_t M, int64_t K, int r) {
+  QuantPlan q;
+  q.row_blocks = ceil_div(M, kQRows);
+  q.chunks = static_cast<int>(K / kQChunk);
+  int64_t want = q.row_blocks > 0 ? ceil_div(kQTargetCtas, q.row_blocks) : 1;
+  if (want < 1) want = 1;
+  if (want > q.chunks) want = q.chunks;
+  q.chunks_per_split = static_cast<int>(ceil_div(q.chunks, want));
+  q.splits = static_cast<int>(ceil_div(q.chunks, q.chunks_per_split));
+  q.off_partials = 0;
+  q.off_tickets = round256(sizeof(float) * kAmaxMaxBlocks);
+  q.off_upart = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks > 0 ? q.row_blocks : 1));
+  const size_t upart = r > 0 ? sizeof(float) * static_cast<size_t>(q.splits) * q.row_blocks * kQRows * 32 : 0;
+  q.bytes = q.off_upart + round256(upart);
+  return q;
+}
+
+bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0 && K <= (int64_t(1) << 30); }
+
+template <typename SrcT>
+int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* inv_s, const void* L1t, int r,
+                 const float* t_w, uint8_t* q, uint8_t* sf, float* t_out, void* U, void* ws,
+                 cudaStream_t stream, DeviceInfo* dev) {
+  const QuantPlan plan = quant_plan(M, K, r);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* partials = reinterpret_cast<float*>(w + plan.off_partials);
+  int* tickets = reinterpret_cast<int*>(w + plan.off_tickets);
+  float* upart = reinterpret_cast<float*>(w + plan.off_upart);
+
+  constexpr int EPV = 16 / sizeof(SrcT);
+  const int64_t vecs = M * (K / EPV);
+  int64_t grid1 = ceil_div(vecs, kAmaxThreads * 4);
+  if (grid1 > kAmaxMaxBlocks) grid1 = kAmaxMaxBlocks;
+  if (grid1 < 1) grid1 = 1;
+  amax_kernel<SrcT><<<static_cast<unsigned>(grid1), kAmaxThreads, 0, stream>>>(
+      X, M, K, ld, inv_s, partials, tickets, static_cast<int>(plan.row_blocks));
+  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+
+  CUtensorMap tm_x, tm_l1;
+  const bool is_bf16 = sizeof(SrcT) == 2;
+  if (!encode_2d(&tm_x, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, X,
+                 static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(ld) * sizeof(SrcT),
+                 is_bf16 ? 64u : 32u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  if (r > 0) {
+    if (!encode_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, static_cast<uint64_t>(K), static_cast<uint64_t>(r),
+                   static_cast<uint64_t>(K) * 2, 64u, static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B))
+      return W4A4_ERR_CUDA;
+  } else {
+    tm_l1 = tm_x;  // unused
+  }
+  QuantParams p;
+  p.M = M;
+  p.K = K;
+  p.inv_s = inv_s;
+  p.partials = partials;
+  p.n_partials = static_cast<int>(grid1);
+  p.t_w = t_w;
+  p.q = q;
+  p.sf = sf;
+  p.t_out = t_out;
+  p.u_part = upart;
+  p.u_out = static_cast<__nv_bfloat16*>(U);
+  p.tickets = tickets;
+  p.chunks_per_split = plan.chunks_per_split;
+  p.splits = plan.splits;
+  p.has_lr = r > 0 ? 1 : 0;
+  p.status = dev->status_ptr;
+  const dim3 grid2(static_cast<unsigned>(plan.row_blocks), static_cast<unsigned>(plan.splits));
+  quant_kernel<SrcT><<<grid2, kQThreads, QuantTile<SrcT>::kSmem, stream>>>(tm_x, tm_l1, p);
+  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  return W4A4_OK;
+}
+
+template <class C>
+int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                    int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                    const void* bias, int epi, void* Y, int64_t ldy, cudaStream_t stream, DeviceInfo* dev) {
+  CUtensorMap ta, tb, tsa, tsb, tu, tl;
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(K / 2), 128u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  if (!encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
+                 static_cast<uint64_t>(K / 2), 128u, static_cast<uint32_t>(C::BN), CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  if (!encode_sf(&tsa, Xsf, M, K, 1)) return W4A4_ERR_CUDA;
+  if (!encode_sf(&tsb, Wsf, N, K, 2)) return W4A4_ERR_CUDA;
+  if (r > 0) {
+    if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, 64u, static_cast<uint64_t>(M), 128u, 64u, 128u,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return W4A4_ERR_CUDA;
+    if (!encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2t, 32u, static_cast<uint64_t>(N), 64u, 32u,
+                   static_cast<uint32_t>(C::BN), CU_TENSOR_MAP_SWIZZLE_64B))
+      return W4A4_ERR_CUDA;
+  } else {
+    tu = ta;
+    tl = ta;
+  }
+  GemmParams p;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.ldy = ldy;
+  p.t_x = t_x;
+  p.t_w = t_w;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.has_lr = r > 0 ? 1 : 0;
+  p.epi = epi;
+  p.status = dev->status_ptr;
+  const int64_t tiles = ceil_div(M, C::BM) * ceil_div(N, C::BN);
+  const int64_t grid = tiles < dev->num_sms ? tiles : dev->num_sms;
+  gemm_kernel<C><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, stream>>>(ta, tb, tsa, tsb, tu, tl, p);
+  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  return W4A4_OK;
+}
+
+int check_gemm_args(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                    int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                    const void* bias, int epi, const void* Y, int64_t ldy) {
+  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || M > (int64_t(1) << 30) || N > (int64_t(1) << 30))
+    return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (epi != W4A4_EPI_NONE && epi != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
+  if (ldy < N || ldy % 8 != 0) return W4A4_ERR_SHAPE;
+  if (!Xq || !Xsf || !t_x || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
+  if (r > 0 && (!U || !L2t)) return W4A4_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(Xsf) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(Y) ||
+      (bias && !aligned16(bias)) || (U && !aligned16(U)) || (L2t && !aligned16(L2t)))
+    return W4A4_ERR_ALIGN;
+  return W4A4_OK;
+}
+
+}  // namespace
+}  // namespace w4a4
+
+using namespace w4a4;
+
+extern "C" {
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 64 != 0) return 0;
+  return static_cast<size_t>(ceil_div(rows, 128)) * 128 * static_cast<size_t>(K / 16);
+}
+
+size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r) {
+  if (M < 0 || !valid_k(K) || (r != 0 && r != 32)) return 0;
+  return quant_plan(M, K, r).bytes;
+}
+
+size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || (r != 0 && r != 32)) return 0;
+  size_t b = quant_plan(M, K, r).bytes;
+  b += round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));  // Xq
+  b += round256(nvfp4_sf_bytes(M, K));                                  // Xsf
+  b += 256;                                                             // t_x
+  b += round256(r > 0 ? static_cast<size_t>(M) * 64 * 2 : 0);           // U hi|lo
+  return b;
+}
+
+int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, const float* inv_s, const void* L1t, int r,
+                       const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;
+  if (r > 0 && (!L1t || !t_w || !U)) return W4A4_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(Xsf) || (inv_s && !aligned16(inv_s)) ||
+      (L1t && !aligned16(L1t)) || (U && !aligned16(U)) || (workspace && !aligned16(workspace)))
+    return W4A4_ERR_ALIGN;
+  if (!workspace || workspace_bytes < nvfp4_quant_workspace_bytes(M, K, r)) return W4A4_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  return launch_quant<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf,
+                                     t_x, U, workspace, static_cast<cudaStream_t>(stream), dev);
+}
+
+int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_t ldr, uint8_t* Wq, uint8_t* Wsf,
+                      float* t_w, void* workspace, size_t workspace_bytes, void* stream) {
+  if (src_dtype != W4A4_SRC_BF16 && src_dtype != W4A4_SRC_F32) return W4A4_ERR_ARG;
+  const int64_t vec = src_dtype == W4A4_SRC_BF16 ? 8 : 4;
+  if (N < 0 || !valid_k(K) || ldr < K || ldr % vec != 0 || N > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
+  if (!R || !Wq || !Wsf || !t_w) return W4A4_ERR_NULL;
+  if (!aligned16(R) || !aligned16(Wq) || !aligned16(Wsf) || (workspace && !aligned16(workspace)))
+    return W4A4_ERR_ALIGN;
+  if (!workspace || workspace_bytes < nvfp4_quant_workspace_bytes(N, K, 0)) return W4A4_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  if (N == 0) return W4A4_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (src_dtype == W4A4_SRC_BF16)
+    return launch_quant<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(R), N, K, ldr, nullptr, nullptr, 0, nullptr,
+                                       Wq, Wsf, t_w, nullptr, workspace, s, dev);
+  return launch_quant<float>(static_cast<const float*>(R), N, K, ldr, nullptr, nullptr, 0, nullptr, Wq, Wsf, t_w,
+                             nullptr, workspace, s, dev);
+}
+
+int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N, int64_t K,
+              const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r, const void* bias,
+              int epilogue, void* Y, int64_t ldy, void* stream) {
+  int st = check_gemm_args(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy);
+  if (st != W4A4_OK) return st;
+  DeviceInfo* dev = nullptr;
+  st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 192-wide tiles (double-buffered accumulator) when N allows, else 256.
+  if (N % 192 == 0)
+    return launch_gemm_cfg<GemmCfg<192, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
+                                            s, dev);
+  return launch_gemm_cfg<GemmCfg<256, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, s,
+                                          dev);
+}
+
+int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,
+                const float* t_w, const float* inv_s, const void* L1t, const void* L2t, int r, const void* bias,
+                int epilogue, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (epilogue != W4A4_EPI_NONE && epilogue != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
+  if (!X || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
+  if (r > 0 && (!L1t || !L2t)) return W4A4_ERR_NULL;
+  if (!workspace || workspace_bytes < w4a4_workspace_bytes(M, N, K, r)) return W4A4_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return W4A4_ERR_ALIGN;
+  const QuantPlan plan = quant_plan(M, K, r);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  size_t off = plan.bytes;
+  uint8_t* Xq = w + off;
+  off += round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
+  uint8_t* Xsf = w + off;
+  off += round256(nvfp4_sf_bytes(M, K));
+  float* t_x = reinterpret_cast<float*>(w + off);
+  off += 256;
+  void* U = r > 0 ? static_cast<void*>(w + off) : nullptr;
+  int st = nvfp4_quantize_act(X, M, K, K, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, workspace, plan.bytes, stream);
+  if (st != W4A4_OK) return st;
+  return w4a4_gemm(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, N, stream);
+}
+
+int w4a4_device_status(int* status, int reset) {
+  if (!status) return W4A4_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+  *status = v;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+  }
+  return W4A4_OK;
+}
+
+const char* w4a4_status_string(int status) {
+  switch (status) {
+    case W4A4_OK: return "ok";
+    case W4A4_ERR_NULL: return "a required pointer is NULL";
+    case W4A4_ERR_SHAPE: return "unsupported size or rank";
+    case W4A4_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
+    case W4A4_ERR_ARCH: return "no CUDA device of compute capability 10.x (sm_100a) is current";
+    case W4A4_ERR_WORKSPACE: return "workspace missing or too small";
+    case W4A4_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case W4A4_ERR_DEVICE_TIMEOUT: return "a device-side pipeline wait exceeded its bound";
+    case W4A4_ERR_ARG: return "an enum argument is out of range";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

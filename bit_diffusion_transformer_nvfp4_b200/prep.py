@@ -1,0 +1,56 @@
+"""Offline SVDQuant preparation of a linear layer's weight (runs once per
+weight, never on the per-step hot path).
+
+Steps ("SVDQuant Guide: 4-Bit DiT Acceleration & Outlier Absorption"):
+1. smoothing factors s_k = max|Xcal_k|^alpha / max|W_k|^(1-alpha), clamped to
+   [1e-4, 1e4] (pillar 2, "SmoothQuant Pre-Conditioning for DiTs"; the
+   SmoothQuant form of s is this library's reading, the page gives only the
+   transform W' = W diag(s), X' = diag(s)^-1 X);
+2. a rank-r factorisation W~ = W diag(s) ~ A~ B~ with the singular values split
+   evenly between the factors (pillar 1 and the page's "Step 1" decomposer),
+   computed here with a randomised truncated SVD;
+3. the residual R = W~ - A~ B~ is packed to NVFP4 by the library's
+   ``nvfp4_pack_weight`` kernel; L1t = B~ diag(1/s) and L2t = A~ are kept in bf16.
+
+Dense linear algebra of this one-off step uses PyTorch's library routines on
+the GPU; the packing itself runs in the library's own kernel.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import PackedWeight, pack_weight
+
+
+def smoothing_factors(x_cal: torch.Tensor, w: torch.Tensor, alpha: float = 0.5) -> torch.Tensor:
+    ax = x_cal.abs().amax(dim=0).double()
+    aw = w.abs().amax(dim=0).double()
+    s = ax.pow(alpha) / aw.pow(1.0 - alpha)
+    ok = (ax > 0) & (aw > 0) & torch.isfinite(s)
+    s = torch.where(ok, s, torch.ones_like(s))
+    return s.clamp(1e-4, 1e4)
+
+
+def svdquant_prepare(w: torch.Tensor, x_cal: torch.Tensor, r: int = 32, alpha: float = 0.5,
+                     bias: torch.Tensor | None = None, niter: int = 2, seed: int = 0) -> PackedWeight:
+    """Prepare one linear (weight [N, K] on the GPU) for ``linear``/``gemm``."""
+    s = smoothing_factors(x_cal, w, alpha)
+    inv_s = (1.0 / s.float()).contiguous()
+    w_s = w.double() * s[None, :]
+    if r > 0:
+        gen_state = torch.random.get_rng_state()
+        torch.manual_seed(seed)
+        u, sv, v = torch.svd_lowrank(w_s, q=min(r + 16, min(w_s.shape)), niter=niter)
+        torch.random.set_rng_state(gen_state)
+        root = sv[:r].sqrt()
+        a = u[:, :r] * root[None, :]            # A~ [N, r]
+        b = root[:, None] * v[:, :r].T          # B~ [r, K]
+        resid = (w_s - a @ b).float().contiguous()
+        L1t = (b / s[None, :]).to(torch.bfloat16).contiguous()
+        L2t = a.to(torch.bfloat16).contiguous()
+    else:
+        resid = w_s.float().contiguous()
+        L1t = L2t = None
+    packed = pack_weight(resid, inv_s=inv_s, L1t=L1t, L2t=L2t,
+                         bias=None if bias is None else bias.to(torch.bfloat16).contiguous())
+    return packed

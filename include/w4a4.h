@@ -1,0 +1,177 @@
+/*
+ * w4a4.h -- C ABI of the B200 (sm_100a) W4A4 NVFP4 linear layer.
+ *
+ * The operation is the dual-branch SVDQuant linear of a diffusion transformer
+ * ("SVDQuant Guide: 4-Bit DiT Acceleration & Outlier Absorption", pillar 1
+ * "Mathematical Outlier Factorization" and pillar 2 "SmoothQuant
+ * Pre-Conditioning for DiTs"; section "Step 2: The SVDQuant Dual-Branch Linear
+ * Layer"), written token-major:
+ *
+ *     Y = bf16( Q(X diag(s)^-1) Q(R)^T  +  (X L1) L2  +  bias )
+ *
+ *   X    [M, K]  bf16 activation, M tokens, K input channels
+ *   s    [K]     smoothing factors (the caller passes inv_s = 1/s in fp32)
+ *   R    [N, K]  residual of the smoothed weight after its rank-r part
+ *   L1   [K, r]  low-rank down-projection, 1/s folded in (passed as L1t = L1^T [r, K])
+ *   L2   [r, N]  low-rank up-projection (passed as L2t = L2^T [N, r])
+ *   Q()  NVFP4 quantisation: E2M1 element codes {0,+-0.5,+-1,+-1.5,+-2,+-3,+-4,+-6},
+ *        one unsigned E4M3 scale per 16 consecutive K elements, one fp32 scale
+ *        per tensor.  NVFP4 is the format the pages name for FLUX on Blackwell
+ *        ("NVIDIA Technical Blog Details FLUX 3 Image Klein Blackwell Inference
+ *        Optimization Methods ...", first optimisation layer); its exact
+ *        arithmetic is fixed below.
+ *
+ * Quantisation arithmetic (every step one correctly rounded fp32 operation):
+ *   x~ = x * inv_s[k];  A = max |x~| over the tensor;
+ *   t = A / 2688 (2688 = 6 * 448), t = 1 if that is not a normal fp32 number;
+ *   per 16-block: b = max |x~|, scale byte e = E4M3_rn_satfinite((b * (1/t)) / 6);
+ *   code = E2M1_rn_satfinite(x~ * (1 / (dec(e) * t))), all +0 if dec(e) == 0.
+ *   Two codes per byte, the even K index in the low nibble.
+ *
+ * Memory layouts (all device memory, row-major unless stated):
+ *   packed codes   [rows, K/2] uint8
+ *   block scales   "SF atom" layout, nvfp4_sf_bytes(rows, K) bytes: rows are
+ *                  grouped in blocks of 128 (the last block padded), K in groups
+ *                  of 64 (4 scales).  Each (128-row block rb, 64-K group kg)
+ *                  pair is a 512-byte atom at offset (rb * K/64 + kg) * 512;
+ *                  inside it, the scale of row m and 16-block j (j = 0..3 in
+ *                  the group) sits at byte (m % 32) * 16 + ((m / 32) % 4) * 4 + j.
+ *                  This is the order in which the tensor cores read scales.
+ *   U (low-rank)   [M, 2r] bf16: columns [0, r) hold hi = bf16(u'), columns
+ *                  [r, 2r) hold lo = bf16(u' - hi), where u' = (X L1) / (t_x t_w)
+ *                  in fp32.  hi + lo carries u' to about 16 significant bits.
+ *
+ * Conventions:
+ *   - The caller owns every buffer.  No function allocates, frees or
+ *     synchronises; all work is enqueued on `stream` (a cudaStream_t, NULL for
+ *     the legacy default stream).  Scalars (t_x, t_w) stay in device memory.
+ *   - Host-detectable problems return an error before anything is enqueued.
+ *   - Pointers must be 16-byte aligned; ldx/ldr/ldy are in elements.
+ *   - Constraints: K % 256 == 0, K >= 256; N % 8 == 0; r in {0, 32};
+ *     M >= 0 (M == 0 is a no-op), rows need not be a multiple of 128.
+ *   - A device-side pipeline wait that exceeds its bound (about two seconds)
+ *     records W4A4_ERR_DEVICE_TIMEOUT in a sticky status word, drains its own
+ *     copies and returns; read it with w4a4_device_status() after a sync.
+ *   - The current CUDA device must be compute capability 10.x (B200 / sm_100a);
+ *     there is no fallback.
+ */
+#ifndef W4A4_H_
+#define W4A4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  W4A4_OK = 0,
+  W4A4_ERR_NULL = -1,           /* a required pointer is NULL */
+  W4A4_ERR_SHAPE = -2,          /* unsupported size or rank */
+  W4A4_ERR_ALIGN = -3,          /* pointer or leading dimension not 16-byte aligned */
+  W4A4_ERR_ARCH = -4,           /* no CUDA device, or not compute capability 10.x */
+  W4A4_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than required */
+  W4A4_ERR_CUDA = -6,           /* a CUDA call or kernel launch failed */
+  W4A4_ERR_DEVICE_TIMEOUT = -7, /* sticky device status: a bounded wait gave up */
+  W4A4_ERR_ARG = -8             /* an enum argument is out of range */
+} w4a4_status;
+
+enum { W4A4_EPI_NONE = 0, W4A4_EPI_GELU_TANH = 1 };
+enum { W4A4_SRC_BF16 = 0, W4A4_SRC_F32 = 1 };
+
+/* Bytes of the SF-atom block-scale buffer for a [rows, K] tensor:
+ * ceil(rows / 128) * 128 * K / 16.  Returns 0 for invalid sizes. */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
+
+/* Workspace bytes needed by nvfp4_quantize_act / nvfp4_pack_weight for an
+ * [M, K] input with rank r (amax partial maxima, low-rank partial sums and
+ * per-row-block counters).  Returns 0 for invalid sizes. */
+size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r);
+
+/* Workspace bytes needed by w4a4_linear: the quantisation workspace plus the
+ * quantised activation (codes, scales, t_x) and the low-rank U buffer. */
+size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/*
+ * nvfp4_quantize_act -- online activation quantisation (smooth, tensor amax,
+ * block scales, codes, packing) fused with the low-rank down-projection.
+ * Activations are quantised afresh at every denoising step because their
+ * outlier channels drift with the timestep ("SVDQuant Guide ...", section
+ * "Why Standard Low-Bit Quantization Fails on DiTs", "Timestep-Dynamic
+ * Activation Drift").
+ *
+ *   X      in   bf16 [M, ldx] row-major, the first K columns are used
+ *   inv_s  in   fp32 [K] reciprocal smoothing factors, NULL = all ones
+ *   L1t    in   bf16 [r, K] (NULL iff r == 0)
+ *   t_w    in   fp32 device scalar, the weight's tensor scale (needed iff r > 0)
+ *   Xq     out  uint8 [M, K/2] packed E2M1 codes
+ *   Xsf    out  uint8 SF-atom layout, nvfp4_sf_bytes(M, K) bytes (pad rows get 0)
+ *   t_x    out  fp32 device scalar, the activation's tensor scale
+ *   U      out  bf16 [M, 2r] hi/lo low-rank activations (NULL iff r == 0)
+ *   workspace   >= nvfp4_quant_workspace_bytes(M, K, r) bytes of device memory,
+ *               contents need not be initialised; must not overlap the outputs
+ * Launches two kernels (tensor amax, then quantise + down-projection).
+ */
+int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx,
+                       const float* inv_s, const void* L1t, int r, const float* t_w,
+                       uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_pack_weight -- offline NVFP4 packing of the residual weight R [N, K]
+ * (bf16 or fp32 source, row stride ldr elements) with the same quantiser
+ * (no smoothing: the smoothing factors are already multiplied into R).  The
+ * pages quantise the residual after removing the low-rank part ("SVDQuant
+ * Guide ...", "Step 1: Low-Rank Outlier Decomposition in PyTorch").
+ *   Wq out uint8 [N, K/2]; Wsf out nvfp4_sf_bytes(N, K) bytes; t_w out fp32 scalar.
+ */
+int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_t ldr,
+                      uint8_t* Wq, uint8_t* Wsf, float* t_w,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * w4a4_gemm -- block-scaled FP4 GEMM on the tcgen05 tensor cores fused with
+ * the low-rank up-projection, bias and the bf16 cast (the fused 4-bit +
+ * low-rank kernel of "SVDQuant Guide ...", pillar 3 "The Nunchaku Fused Kernel
+ * Engine", re-designed for sm_100a):
+ *   Y[m,n] = bf16( t_x t_w ( sum_k dec(Xq) dec(Xsf) dec(Wq) dec(Wsf)
+ *                            + sum_j U[m,j] L2t[n,j] ) + bias[n] )
+ * with U the hi/lo pair written by nvfp4_quantize_act (so the low-rank term is
+ * (X L1) L2 after the t_x t_w factor).  epilogue = W4A4_EPI_GELU_TANH applies
+ * 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) before the bf16 cast.
+ *   Xq/Xsf/t_x/U  in  as written by nvfp4_quantize_act (U NULL iff r == 0)
+ *   Wq/Wsf/t_w    in  as written by nvfp4_pack_weight
+ *   L2t  in  bf16 [N, r] (NULL iff r == 0);  bias in bf16 [N] or NULL
+ *   Y    out bf16 [M, ldy], ldy >= N, ldy % 8 == 0
+ */
+int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U,
+              int64_t M, int64_t N, int64_t K,
+              const uint8_t* Wq, const uint8_t* Wsf, const float* t_w,
+              const void* L2t, int r, const void* bias, int epilogue,
+              void* Y, int64_t ldy, void* stream);
+
+/*
+ * w4a4_linear -- the whole hot path: nvfp4_quantize_act on X (row stride K)
+ * into the workspace, then w4a4_gemm into Y (row stride N).
+ *   workspace >= w4a4_workspace_bytes(M, N, K, r) bytes of device memory.
+ */
+int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K,
+                const uint8_t* Wq, const uint8_t* Wsf, const float* t_w,
+                const float* inv_s, const void* L1t, const void* L2t, int r,
+                const void* bias, int epilogue, void* Y,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Copies the sticky device status word of the current device into *status
+ * (W4A4_OK or W4A4_ERR_DEVICE_TIMEOUT) and clears it if reset != 0.  This call
+ * synchronises the device.  Returns W4A4_OK or W4A4_ERR_CUDA. */
+int w4a4_device_status(int* status, int reset);
+
+/* Static description of a status code; never NULL. */
+const char* w4a4_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A4_H_ */

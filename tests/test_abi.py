@@ -1,0 +1,86 @@
+"""The C ABI library: it builds, loads, exports every declared symbol, and its
+host-side checks reject bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a4.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in {"if", "defined"}))
+
+
+@pytest.fixture(scope="module")
+def so():
+    from bit_diffusion_transformer_nvfp4_b200 import build
+    build.build()
+    import bit_diffusion_transformer_nvfp4_b200 as w
+    return w.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["nvfp4_quantize_act", "nvfp4_pack_weight", "w4a4_gemm", "w4a4_linear", "nvfp4_sf_bytes",
+              "nvfp4_quant_workspace_bytes", "w4a4_workspace_bytes", "w4a4_device_status",
+              "w4a4_status_string"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(so):
+    for n in declared_functions():
+        assert hasattr(so, n), n
+        assert isinstance(getattr(so, n), ctypes._CFuncPtr)
+
+
+def test_sizes(so):
+    assert so.nvfp4_sf_bytes(300, 512) == 384 * 32
+    assert so.nvfp4_sf_bytes(128, 3072) == 128 * 192
+    assert so.nvfp4_sf_bytes(0, 256) == 0
+    assert so.nvfp4_sf_bytes(10, 100) == 0
+    assert so.nvfp4_quant_workspace_bytes(4608, 3072, 32) > 4608 * 32 * 4
+    assert so.nvfp4_quant_workspace_bytes(4608, 3000, 32) == 0
+    assert so.nvfp4_quant_workspace_bytes(4608, 3072, 16) == 0
+    ws = so.w4a4_workspace_bytes(4608, 9216, 3072, 32)
+    assert ws >= 4608 * 1536 + 4608 * 192 + 4608 * 128
+    assert so.w4a4_workspace_bytes(4608, 9210, 3072, 32) == 0
+
+
+def test_status_strings(so):
+    for st in range(-8, 1):
+        assert so.w4a4_status_string(st)
+    assert so.w4a4_status_string(-7) == b"a device-side pipeline wait exceeded its bound"
+
+
+def test_host_validation_before_any_launch(so):
+    import bit_diffusion_transformer_nvfp4_b200 as w
+    P = 1 << 20  # aligned fake device address, never dereferenced
+    big = 1 << 30
+    q = w.lib().nvfp4_quantize_act
+    assert q(None, 128, 512, 512, None, None, 0, None, P, P, P, None, P, big, None) == -1     # NULL X
+    assert q(P, 128, 500, 512, None, None, 0, None, P, P, P, None, P, big, None) == -2        # K % 256
+    assert q(P, 128, 512, 500, None, None, 0, None, P, P, P, None, P, big, None) == -2        # ldx < K
+    assert q(P, 128, 512, 512, None, None, 16, None, P, P, P, None, P, big, None) == -2       # rank
+    assert q(P, 128, 512, 512, None, None, 32, None, P, P, P, None, P, big, None) == -1       # no L1t
+    assert q(P + 2, 128, 512, 512, None, None, 0, None, P, P, P, None, P, big, None) == -3    # alignment
+    assert q(P, 128, 512, 512, None, None, 0, None, P, P, P, None, P, 16, None) == -5         # workspace
+    g = w.lib().w4a4_gemm
+    assert g(P, P, P, None, 128, 100, 512, P, P, P, None, 0, None, 0, P, 100, None) == -2     # N % 8
+    assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 7, P, 128, None) == -8     # epilogue
+    assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 120, None) == -2     # ldy < N
+    assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 32, None, 0, P, 128, None) == -1    # no U/L2t
+    pw = w.lib().nvfp4_pack_weight
+    assert pw(P, 5, 128, 512, 512, P, P, P, P, big, None) == -8                               # dtype
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU path")
+def test_no_gpu_reports_arch_error(so):
+    P = 1 << 20
+    st = so.nvfp4_quantize_act(P, 128, 512, 512, None, None, 0, None, P, P, P, None, P, 1 << 30, None)
+    assert st == -4
