@@ -277,7 +277,7 @@ def run_ours(args):
         "wall_s_timed": round(t_wall1 - t_wall0, 3),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(case, sample_rows=args.cpu_rows)
+        out["cpu_baseline"] = cpu_baseline(case, args.cpu_rows, args.cpu_cols)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -296,27 +296,48 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def oracle_prepared(case):
+def oracle_prepared(case, cols):
+    """Oracle-side preparation (not timed): smoothing, SVD, and the NVFP4
+    packing of the weight rows of the sampled output channels under the whole
+    residual's tensor scale."""
     from oracle import nvfp4, prep
     p = prep.svdquant_prepare(case.w, case.x_cal, case.r, case.alpha)
-    wq, wsf, tw, _ = nvfp4.quantize_activation(p["R"], None)
-    return p, wq, wsf, tw
+    R = p["R"]
+    codes, wsf, tw, _ = nvfp4.quantize(R[cols], amax=np.max(np.abs(R)))
+    return p, nvfp4.pack(codes), wsf, tw
 
 
-def cpu_baseline(case, sample_rows=512, prepared=None):
-    """The oracle as it stands on a bounded sample: the whole activation is
-    quantised (the tensor scale needs every row) and Y is formed for
-    ``sample_rows`` rows; throughput counts the sampled rows' FLOPs."""
+def sample_indices(case, rows, cols):
+    g = np.random.Generator(np.random.PCG64(7))
+    return (np.sort(g.choice(case.M, rows, replace=False)), np.sort(g.choice(case.N, cols, replace=False)))
+
+
+def oracle_step(case, prepared, rows, cols):
     from oracle import linear as olinear
-    p, wq, wsf, tw = prepared or oracle_prepared(case)
-    rows = np.sort(np.random.Generator(np.random.PCG64(7)).choice(case.M, sample_rows, replace=False))
+    p, wq, wsf, tw = prepared
+    olinear.w4a4_linear(case.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"][cols],
+                        None if case.bias is None else case.bias[cols], rows=rows)
+
+
+def cpu_baseline(case, n_rows=1024, n_cols=2048, min_seconds=10.0):
+    """The oracle as it stands on a bounded sample of the workload: the whole
+    activation's tensor scale, then quantisation of ``n_rows`` sampled tokens
+    and Y for them on ``n_cols`` sampled output channels (numpy fp32
+    quantiser, fp64 matmul).  Throughput counts the sample's FLOPs."""
+    rows, cols = sample_indices(case, n_rows, n_cols)
+    prepared = oracle_prepared(case, cols)
+    iters = 0
     t0 = time.perf_counter()
-    olinear.w4a4_linear(case.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"], case.bias, rows=rows)
-    dt = time.perf_counter() - t0
-    fl = flops_per_step(sample_rows, case.K, case.N, case.r)
+    while True:
+        oracle_step(case, prepared, rows, cols)
+        iters += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds:
+            break
+    fl = flops_per_step(n_rows, case.K, n_cols, case.r) * iters
     return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"whole-tensor activation quantisation + Y for {sample_rows} of {case.M} rows "
-                      f"(numpy fp32 quantiser, fp64 matmul), {dt:.2f} s"}
+            "sample": f"{n_rows} of {case.M} tokens x {n_cols} of {case.N} output channels, K={case.K}, "
+                      f"whole-tensor activation scale; repeated {iters}x in {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -325,22 +346,24 @@ def run_reference(args):
         return
     from synth import config_cases
     case = config_cases(2)[0]
-    prepared = oracle_prepared(case)
-    rows = args.ref_rows
+    rows, cols = sample_indices(case, args.ref_rows, args.ref_cols)
+    prepared = oracle_prepared(case, cols)
     for _ in range(args.warmup):
-        cpu_baseline(case, rows, prepared)
+        oracle_step(case, prepared, rows, cols)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        cpu_baseline(case, rows, prepared)
+        oracle_step(case, prepared, rows, cols)
     dt = time.perf_counter() - t0
-    fl = flops_per_step(rows, case.K, case.N, case.r)
+    fl = flops_per_step(args.ref_rows, case.K, args.ref_cols, case.r)
     value = fl * args.steps / dt / 1e12
+    sample = (f"per step: {args.ref_rows} of {case.M} tokens x {args.ref_cols} of {case.N} output channels, "
+              f"K={case.K}, whole-tensor activation scale")
     out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": 0,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": dict(WORKLOAD, parallelism="host CPU"),
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cpu_threads(), "kind": "oracle",
-                            "sample": f"per step: whole-tensor activation quantisation + Y for {rows} of {case.M} rows"},
+                            "sample": sample},
            "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -351,8 +374,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-rows", type=int, default=512)
-    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-rows", type=int, default=1024)
+    ap.add_argument("--cpu-cols", type=int, default=2048)
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--ref-cols", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

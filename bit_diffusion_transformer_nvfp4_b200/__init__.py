@@ -165,6 +165,19 @@ class PackedWeight:
         self.inv_s, self.L1t, self.L2t, self.bias = inv_s, L1t, L2t, bias
         self.r = 0 if L1t is None else int(L1t.shape[0])
 
+    def rows(self, r0: int, r1: int) -> "PackedWeight":
+        """Views of output channels [r0, r1) (r0 a multiple of 128): the same
+        activation quantisation (smoothing, L1t, t_w) serves both parts of a
+        fused projection."""
+        if r0 % 128 or not (0 <= r0 < r1 <= self.N):
+            raise ValueError("row slice must start on a 128-row boundary")
+        atom_row = (self.K // 64) * 512
+        sf0 = (r0 // 128) * atom_row
+        sf1 = -(-r1 // 128) * atom_row
+        return PackedWeight(self.Wq[r0:r1], self.Wsf[sf0:sf1], self.t_w, r1 - r0, self.K, self.inv_s,
+                            self.L1t, None if self.L2t is None else self.L2t[r0:r1],
+                            None if self.bias is None else self.bias[r0:r1])
+
 
 def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None) -> QuantizedActivation:
     M, K = X.shape

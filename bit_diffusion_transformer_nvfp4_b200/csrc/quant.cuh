@@ -31,7 +31,10 @@ constexpr int kAmaxThreads = 256;
 constexpr int kAmaxMaxBlocks = 1024;
 constexpr int kQRows = 128;       // rows per CTA (one TMEM lane per row)
 constexpr int kQChunk = 64;       // K elements per pipeline step (one SF atom column)
-constexpr int kQThreads = 128;
+constexpr int kQComputeWarps = 4;  // one thread per row of the 128-row tile
+constexpr int kQProducerWarp = 4;  // TMA producer
+constexpr int kQMmaWarp = 5;       // TMEM owner, issues the U = X L1 MMAs
+constexpr int kQThreads = 32 * 6;
 constexpr int kQTargetCtas = 296; // two CTAs per SM on a 148-SM part
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -53,11 +56,10 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restri
   const int64_t total = M * vec_per_row;
   float m = 0.0f;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i < total; i += stride) {
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  auto absmax_vec = [&](int64_t i, const uint4 raw) {
     const int64_t row = i / vec_per_row;
     const int64_t col = (i - row * vec_per_row) * EPV;
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(X + row * ld + col));
     float v[EPV];
     if constexpr (sizeof(SrcT) == 2) {
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -84,7 +86,22 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restri
     }
 #pragma unroll
     for (int j = 0; j < EPV; ++j) m = fmaxf(m, fabsf(v[j]));
+  };
+  auto load = [&](int64_t i) {
+    const int64_t row = i / vec_per_row;
+    const int64_t col = (i - row * vec_per_row) * EPV;
+    return __ldcs(reinterpret_cast<const uint4*>(X + row * ld + col));
+  };
+  int64_t i = i0;
+  // four independent 16-byte loads in flight per thread
+  for (; i + 3 * stride < total; i += 4 * stride) {
+    const uint4 a = load(i), b = load(i + stride), c = load(i + 2 * stride), d = load(i + 3 * stride);
+    absmax_vec(i, a);
+    absmax_vec(i + stride, b);
+    absmax_vec(i + 2 * stride, c);
+    absmax_vec(i + 3 * stride, d);
   }
+  for (; i < total; i += stride) absmax_vec(i, load(i));
   __shared__ float red[kAmaxThreads / 32];
   m = warp_max(m);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -125,8 +142,11 @@ struct QuantTile {
   static constexpr int kBoxes = sizeof(SrcT) / 2;
   static constexpr int kStages = sizeof(SrcT) == 2 ? 4 : 3;
   static constexpr int kL1Bytes = 32 * kQChunk * 2;  // L1t tile, 32 x 64 bf16 (4 KB)
-  static constexpr int kStageBytes = kBytes + (sizeof(SrcT) == 2 ? kL1Bytes : 0);
+  static constexpr int kL1Off = kBytes;
+  static constexpr int kInvSOff = kBytes + (sizeof(SrcT) == 2 ? kL1Bytes : 0);  // 64 fp32 of inv_s
+  static constexpr int kStageBytes = (kInvSOff + kQChunk * 4 + 1023) / 1024 * 1024;
   static constexpr int kSmem = kStageBytes * kStages + 1024 + 256;
+  static_assert(kStageBytes * kStages + 8 * (3 * kStages + 1) + 64 <= kStageBytes * kStages + 256, "barrier area");
 };
 
 // Read 8 consecutive source elements [8c, 8c+8) of row ``r`` from a 128-byte
@@ -159,7 +179,7 @@ __device__ __forceinline__ float tensor_scale_from(float amax) {
 }
 
 template <typename SrcT>
-__global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant__ CUtensorMap tm_x,
+__global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                           const __grid_constant__ CUtensorMap tm_l1,
                                                           const QuantParams p) {
   using Tile = QuantTile<SrcT>;
@@ -167,14 +187,17 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tile::kStageBytes * S);
-  uint64_t* mma_done = full + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + S);
+  uint64_t* empty = full + S;
+  uint64_t* mma_done = empty + S;
+  uint64_t* drain = mma_done + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 4 floats
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 6);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 6 floats
+  int* last_flag = reinterpret_cast<int*>(tmem_slot + 8);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int rb = blockIdx.x;
   const int split = blockIdx.y;
   const int chunks = static_cast<int>(p.K / kQChunk);
@@ -186,66 +209,95 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant_
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), kQComputeWarps);
       mbar_init(smem_u32(&mma_done[s]), 1);
     }
+    mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tm_x);
-    if (lr) tma_prefetch_desc(&tm_l1);
   }
-  if (lr && warp == 0) {
+  if (lr && warp == kQMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 32);
     tmem_relinquish();
   }
-  // tensor scale from the pass-1 partial maxima (same value in every CTA)
+  // tensor scale from the pass-1 partial maxima (the same value in every CTA)
   float m = 0.0f;
   for (int i = tid; i < p.n_partials; i += kQThreads) m = fmaxf(m, p.partials[i]);
   m = warp_max(m);
-  if ((tid & 31) == 0) red[warp] = m;
+  if (lane == 0) red[warp] = m;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const float amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float amax = red[0];
+#pragma unroll
+  for (int w = 1; w < kQThreads / 32; ++w) amax = fmaxf(amax, red[w]);
   const float t = tensor_scale_from(amax);
   const float rt = __frcp_rn(t);
   if (rb == 0 && split == 0 && tid == 0) *p.t_out = t;
   const uint32_t tmem = lr ? *tmem_slot : 0u;
 
-  auto issue = [&](int i) {
-    const int s = i % S;
-    const uint32_t bar = smem_u32(&full[s]);
-    uint8_t* dst = smem + s * Tile::kStageBytes;
-    const int kx = (kc0 + i) * kQChunk;
-    if constexpr (sizeof(SrcT) == 2) {
-      mbar_arrive_expect_tx(bar, Tile::kBytes + (lr ? Tile::kL1Bytes : 0));
-      tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
-      if (lr) tma_load_2d(smem_u32(dst + Tile::kBytes), &tm_l1, bar, kx, 0);
-    } else {
-      mbar_arrive_expect_tx(bar, Tile::kBytes);
-      tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
-      tma_load_2d(smem_u32(dst + kQRows * 128), &tm_x, bar, kx + 32, rb * kQRows);
+  if (warp == kQProducerWarp) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_x);
+      if (lr) tma_prefetch_desc(&tm_l1);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int s = i % S;
+        if (i >= S) {
+          const uint32_t ph = ((i / S) - 1) & 1;   // the fill of chunk i - S
+          if (!mbar_wait(smem_u32(&empty[s]), ph, abort_flag, p.status)) break;
+          if (lr && !mbar_wait(smem_u32(&mma_done[s]), ph, abort_flag, p.status)) break;
+        }
+        const uint32_t bar = smem_u32(&full[s]);
+        uint8_t* dst = smem + s * Tile::kStageBytes;
+        const int kx = (kc0 + i) * kQChunk;
+        const uint32_t inv_bytes = p.inv_s != nullptr ? kQChunk * 4 : 0;
+        if constexpr (sizeof(SrcT) == 2) {
+          mbar_arrive_expect_tx(bar, Tile::kBytes + (lr ? Tile::kL1Bytes : 0) + inv_bytes);
+          tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
+          if (lr) tma_load_2d(smem_u32(dst + Tile::kL1Off), &tm_l1, bar, kx, 0);
+        } else {
+          mbar_arrive_expect_tx(bar, Tile::kBytes + inv_bytes);
+          tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
+          tma_load_2d(smem_u32(dst + kQRows * 128), &tm_x, bar, kx + 32, rb * kQRows);
+        }
+        if (inv_bytes) bulk_load(smem_u32(dst + Tile::kInvSOff), p.inv_s + kx, inv_bytes, bar);
+        ++issued;
+      }
+      // every fill issued must land before the shared memory is released
+      for (int j = max(0, issued - S); j < issued; ++j) mbar_wait_drain(smem_u32(&full[j % S]), (j / S) & 1);
     }
-  };
-
-  int issued = 0;      // fills issued (thread 0's count)
-  int mma_batches = 0; // low-rank MMA batches committed (thread 0's count)
-  if (tid == 0) {
-    for (; issued < min(S, n); ++issued) issue(issued);
-  }
-
-  const int row_in_tile = tid;
-  const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-  const bool row_ok = row < p.M;
-  const int64_t kbytes = p.K / 2;
-  int consumed = 0;
-  bool aborted = false;
-
-  for (int i = 0; i < n; ++i) {
-    const int s = i % S;
-    const uint32_t ph = (i / S) & 1;
-    const bool ok = mbar_wait(smem_u32(&full[s]), ph, abort_flag, p.status);
-    if (ok) {
-      consumed = i + 1;
+  } else if (warp == kQMmaWarp) {
+    // ------------------------------------------------------- U = X L1 MMAs
+    if (lr && lane == 0) {
+      for (int i = 0; i < n; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(smem_u32(&full[s]), (i / S) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * Tile::kStageBytes);
+        const uint32_t b_base = a_base + Tile::kL1Off;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
+          mma_bf16(tmem, ad, bd, idesc_bf16(128, 32), (i > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&mma_done[s]));
+      }
+      // all MMAs of this thread complete before TMEM is read or released
+      tc_commit(smem_u32(drain));
+      mbar_wait_drain(smem_u32(drain), 0);
+    }
+  } else {
+    // ------------------------------------------------------- quantise rows
+    const int row_in_tile = tid;  // compute warps are warps 0..3
+    const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
+    const bool row_ok = row < p.M;
+    const int64_t kbytes = p.K / 2;
+    for (int i = 0; i < n; ++i) {
+      const int s = i % S;
+      if (!mbar_wait(smem_u32(&full[s]), (i / S) & 1, abort_flag, p.status)) break;
       const uint8_t* tile = smem + s * Tile::kStageBytes;
       const int kc = kc0 + i;
       const int k0 = kc * kQChunk;
@@ -259,26 +311,36 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant_
         for (int j = 0; j < 8; ++j) x[8 * c + j] = v[j];
       }
       if (p.inv_s != nullptr) {
+        const float4* inv = reinterpret_cast<const float4*>(tile + Tile::kInvSOff);
 #pragma unroll
         for (int j = 0; j < 64; j += 4) {
-          const float4 sv = __ldg(reinterpret_cast<const float4*>(p.inv_s + k0 + j));
+          const float4 sv = inv[j / 4];
           x[j] = __fmul_rn(x[j], sv.x);
           x[j + 1] = __fmul_rn(x[j + 1], sv.y);
           x[j + 2] = __fmul_rn(x[j + 2], sv.z);
           x[j + 3] = __fmul_rn(x[j + 3], sv.w);
         }
       }
-      // four 16-element blocks: scale bytes and codes
+      // four 16-element blocks: maxima first (this consumes every value read
+      // from the stage), then release the stage: the shared-memory reads are
+      // ordered before the refill's TMA writes by the proxy fence and the
+      // barrier's release/acquire.
+      float bmx[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float bm = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) bm = fmaxf(bm, fabsf(x[16 * b + j]));
+        bmx[b] = bm;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
       uint32_t sf_word = 0;
       uint32_t codes[8];
 #pragma unroll
       for (int b = 0; b < 4; b += 2) {
-        float bm0 = 0.0f, bm1 = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          bm0 = fmaxf(bm0, fabsf(x[16 * b + j]));
-          bm1 = fmaxf(bm1, fabsf(x[16 * (b + 1) + j]));
-        }
+        const float bm0 = bmx[b], bm1 = bmx[b + 1];
         const float s0 = __fdiv_rn(__fmul_rn(bm0, rt), 6.0f);
         const float s1 = __fdiv_rn(__fmul_rn(bm1, rt), 6.0f);
         const uint32_t e2 = cvt_e4m3x2(s1, s0);  // byte 0 = block b, byte 1 = block b+1
@@ -314,62 +376,26 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant_
                                                     (row_in_tile >> 5) * 4);
         *sfw = sf_word;
       }
-      if (lr && tid == 0) {
-        tc_fence_after();
-        const uint32_t a_base = smem_u32(tile);
-        const uint32_t b_base = smem_u32(tile + Tile::kBytes);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
-          mma_bf16(tmem, ad, bd, idesc_bf16(128, 32), (i > 0 || k > 0) ? 1u : 0u);
-        }
-        tc_commit(smem_u32(&mma_done[s]));
-        ++mma_batches;
-      }
-    }
-    // every thread has finished reading stage s (or somebody gave up)
-    if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
-    if (tid == 0 && issued < n) {
-      // the MMA batch just committed reads stage s; let it finish first
-      if (!lr || mbar_wait(smem_u32(&mma_done[s]), ph, abort_flag, p.status)) {
-        issue(issued);
-        ++issued;
-      }
     }
   }
 
-  if (aborted) {
-    // Drain: wait (bounded) for every TMA fill still in flight and for the
-    // newest low-rank MMA batch, then release TMEM and leave.
-    if (tid == 0) {
-      for (int j = consumed; j < issued; ++j) mbar_wait_drain(smem_u32(&full[j % S]), (j / S) & 1);
-      if (mma_batches > 0) {
-        const int L = mma_batches - 1;
-        mbar_wait_drain(smem_u32(&mma_done[L % S]), (L / S) & 1);
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (lr && warp == 0) {
+  // Every role has finished (or given up); in-flight copies and MMAs drained.
+  tc_fence_before();
+  __syncthreads();
+  const bool aborted = *abort_flag != 0;
+  if (!lr || aborted) {
+    if (lr && warp == kQMmaWarp) {
       tc_fence_after();
       tmem_dealloc(tmem, 32);
     }
     return;
   }
 
-  if (lr) {
-    // U partial of this K slice: wait for the last MMA batch, read TMEM
-    bool ok = true;
-    if (n > 0) {
-      const int s = (n - 1) % S;
-      const uint32_t ph = ((n - 1) / S) & 1;
-      ok = mbar_wait(smem_u32(&mma_done[s]), ph, abort_flag, p.status);
-    }
-    if (__syncthreads_or(!ok)) {
-      if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 32); }
-      return;
-    }
+  // U partial of this K slice (TMEM lane = row): compute warps read it out.
+  const int row_in_tile = tid;
+  const int64_t rows_pad = static_cast<int64_t>(gridDim.x) * kQRows;
+  const int64_t prow = static_cast<int64_t>(rb) * kQRows + row_in_tile;
+  if (warp < kQComputeWarps) {
     tc_fence_after();
     uint32_t u[32];
     tmem_ld_32cols(tmem + (static_cast<uint32_t>(warp * 32) << 16), u);
@@ -378,54 +404,72 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const __grid_constant_
 #pragma unroll
       for (int j = 0; j < 32; ++j) u[j] = 0u;
     }
-    const int64_t prow = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-    const int64_t rows_pad = static_cast<int64_t>(gridDim.x) * kQRows;
     float4* dst = reinterpret_cast<float4*>(p.u_part + (static_cast<int64_t>(split) * rows_pad + prow) * 32);
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       dst[j] = make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
                            __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
     __threadfence();
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) { tc_fence_after(); tmem_dealloc(tmem, 32); }
-    if (tid == 0) {
-      const int ticket = atomicAdd(&p.tickets[rb], 1);
-      *last_flag = (ticket == p.splits - 1) ? 1 : 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kQMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+  if (tid == 0) {
+    const int ticket = atomicAdd(&p.tickets[rb], 1);
+    *last_flag = (ticket == p.splits - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (*last_flag && warp < kQComputeWarps) {
+    // the last K slice of this row block sums the partials in slice order
+    __threadfence();
+    const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
+    float acc[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+    for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
+      // the loads of two slices are in flight together; the sums still run
+      // in slice order
+      float4 w[2][8];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (sp0 + q < p.splits) {
+          const float4* src =
+              reinterpret_cast<const float4*>(p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow) * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[q][j] = __ldcg(src + j);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (sp0 + q < p.splits) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            acc[4 * j] = __fadd_rn(acc[4 * j], w[q][j].x);
+            acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], w[q][j].y);
+            acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], w[q][j].z);
+            acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], w[q][j].w);
+          }
+        }
+      }
     }
-    __syncthreads();
-    if (*last_flag) {
-      __threadfence();
-      float acc[32];
+    if (row < p.M) {
+      const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
+      uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
-      for (int sp = 0; sp < p.splits; ++sp) {
-        const float4* src = reinterpret_cast<const float4*>(p.u_part + (static_cast<int64_t>(sp) * rows_pad + prow) * 32);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 w = __ldcg(src + j);
-          acc[4 * j] = __fadd_rn(acc[4 * j], w.x);
-          acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], w.y);
-          acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], w.z);
-          acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], w.w);
-        }
+      for (int j = 0; j < 32; j += 2) {
+        const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
+        const uint32_t h = pack_bf16x2(a0, a1);
+        hi[j / 2] = h;
+        lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
       }
-      if (row_ok) {
-        const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
-        uint32_t hi[16], lo[16];
+      uint4* dst2 = reinterpret_cast<uint4*>(p.u_out + row * 64);
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
-          const uint32_t h = pack_bf16x2(a0, a1);
-          hi[j / 2] = h;
-          lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
-        }
-        uint4* dst2 = reinterpret_cast<uint4*>(p.u_out + row * 64);
+      for (int j = 0; j < 4; ++j) dst2[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) dst2[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dst2[4 + j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
-      }
+      for (int j = 0; j < 4; ++j) dst2[4 + j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
     }
   }
 }

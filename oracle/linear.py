@@ -37,13 +37,18 @@ def w4a4_linear(x_bf16_as_f32, inv_s, Wq_packed, Wsf, t_w, L1t, L2t, bias=None,
     L1t [r, K], L2t [N, r]  low-rank factors (bf16 values as fp32), r may be 0
     bias [N] or None
     rows          optional row indices: evaluate only these rows of Y.  The
-                  activation scale still comes from the whole tensor.
-    Returns (Y fp64, dict of the activation quantisation results).
+                  activation scale still comes from the whole tensor; only the
+                  selected rows are quantised (rows are independent once the
+                  tensor scale is fixed).
+    The weight arguments may hold a subset of the output channels (with the
+    matching L2t rows and bias entries); Y then has those columns only.
+    Returns (Y fp64, dict of the activation quantisation results of the
+    evaluated rows).
     """
     x = np.asarray(x_bf16_as_f32, np.float32)
-    xq, xsf, t_x, amax = nvfp4.quantize_activation(x, inv_s)
+    xq, xsf, t_x, amax = nvfp4.quantize_activation(x, inv_s, rows)
     sel = slice(None) if rows is None else np.asarray(rows)
-    xdeq = nvfp4.dequantize(nvfp4.unpack(xq[sel]), xsf[sel], t_x)
+    xdeq = nvfp4.dequantize(nvfp4.unpack(xq), xsf, t_x)
     wdeq = nvfp4.dequantize(nvfp4.unpack(Wq_packed), Wsf, t_w)
     y = xdeq @ wdeq.T
     if L1t is not None and np.asarray(L1t).shape[0] > 0:

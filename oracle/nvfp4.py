@@ -164,17 +164,22 @@ def tensor_scale(amax: np.float32) -> np.float32:
     return t
 
 
-def quantize(xs: np.ndarray):
+def quantize(xs: np.ndarray, amax=None):
     """Quantise an already-smoothed fp32 matrix [rows, K] to NVFP4.
 
-    Returns ``(codes u8 [rows, K], sf u8 [rows, K/16], t f32, amax f32)``;
-    codes are unpacked (one per byte, see ``pack``).
+    ``amax`` is the tensor's absolute maximum; when the rows given are a
+    subset of a larger tensor, pass the whole tensor's maximum (once the
+    tensor scale is fixed, every row is quantised independently of the
+    others).  Returns ``(codes u8 [rows, K], sf u8 [rows, K/16], t f32,
+    amax f32)``; codes are unpacked (one per byte, see ``pack``).
     """
     xs = np.asarray(xs, dtype=np.float32)
     rows, K = xs.shape
     if K % BLOCK:
         raise ValueError("K must be a multiple of 16")
-    amax = F32(np.max(np.abs(xs))) if xs.size else F32(0.0)
+    if amax is None:
+        amax = F32(np.max(np.abs(xs))) if xs.size else F32(0.0)
+    amax = F32(amax)
     t = tensor_scale(amax)
     rt = F32(F32(1.0) / t)
     blocks = xs.reshape(rows, K // BLOCK, BLOCK)
@@ -214,8 +219,16 @@ def dequantize(codes: np.ndarray, sf: np.ndarray, t) -> np.ndarray:
     return v.reshape(rows, K)
 
 
-def quantize_activation(x_bf16_as_f32: np.ndarray, inv_s: np.ndarray | None):
-    """Smooth, then quantise.  Returns (packed codes, sf, t, amax)."""
+def quantize_activation(x_bf16_as_f32: np.ndarray, inv_s: np.ndarray | None, rows=None):
+    """Smooth, then quantise.  Returns (packed codes, sf, t, amax).
+
+    With ``rows`` (indices), only those rows are quantised, under the tensor
+    scale of the whole matrix.
+    """
     xs = smooth(x_bf16_as_f32, inv_s)
-    codes, sf, t, amax = quantize(xs)
+    if rows is None:
+        codes, sf, t, amax = quantize(xs)
+    else:
+        amax = F32(np.max(np.abs(xs))) if xs.size else F32(0.0)
+        codes, sf, t, amax = quantize(xs[np.asarray(rows)], amax=amax)
     return pack(codes), sf, t, amax

@@ -31,11 +31,18 @@ def rng(seed: int) -> np.random.Generator:
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
-    """float32 -> bf16 bit patterns, round to nearest even (finite inputs)."""
+    """float32 -> bf16 bit patterns, round to nearest even (finite inputs).
+
+    Uses torch's (multi-threaded, round-to-nearest-even) cast when torch is
+    importable, else the same rounding on the bit pattern in numpy."""
     f = np.ascontiguousarray(np.asarray(a, np.float32))
-    u = f.view(np.uint32)
-    lsb = (u >> 16) & np.uint32(1)
-    return ((u + np.uint32(0x7FFF) + lsb) >> 16).astype(np.uint16)
+    try:
+        import torch
+        return torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    except ImportError:
+        u = f.view(np.uint32)
+        lsb = (u >> 16) & np.uint32(1)
+        return ((u + np.uint32(0x7FFF) + lsb) >> 16).astype(np.uint16)
 
 
 def bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -102,8 +102,9 @@ def test_quant_lowrank_u(w4):
     # relative, 1.4e-6 at K = 512) plus the hi|lo representation (2^-17)
     assert olinear.rel_frobenius(got, ref) < 1e-5
     assert np.max(np.abs(got - ref)) <= 5e-5 * np.max(np.abs(ref))
-    # hi is the bf16 rounding of hi + lo
-    assert np.array_equal(bf16_round((hi + lo).astype(np.float32)), hi)
+    # hi holds the leading bf16 part: |lo| is at most half a bf16 ulp of hi
+    # (plus lo's own rounding)
+    assert np.all(np.abs(lo) <= np.abs(hi) * 2.0 ** -8 * (1 + 2.0 ** -7))
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
@@ -130,3 +131,21 @@ def test_pack_weight(w4, src):
     assert float(pw.t_w.cpu()[0]) == float(ot)
     np.testing.assert_array_equal(wsf[:c.N], osf)
     np.testing.assert_array_equal(wq, oq)
+
+
+@pytest.mark.parametrize("M,K", [(4608, 3072), (1024, 12288)])
+def test_quant_lowrank_stage_reuse(w4, M, K):
+    """Enough K per CTA that the TMA ring stages are refilled while the
+    low-rank MMAs also read them: codes bit-exact and identical run to run."""
+    import torch
+    c = make_linear("t", M, K, 256, r=32, act="normal_outliers", n_out=8, out_scale=60.0, seed=M + K)
+    p = prepare(c)
+    X = to_dev_bf16(c.x)
+    args = (to_dev_f32(p["inv_s"]), to_dev_bf16(p["L1t"]), to_dev_f32(np.array([p["t_w"]], np.float32)))
+    qa = w4.quantize_act(X, *args)
+    qb = w4.quantize_act(X, *args)
+    torch.cuda.synchronize()
+    assert w4.w4a4_device_status() == 0
+    assert torch.equal(qa.Xq, qb.Xq) and torch.equal(qa.Xsf, qb.Xsf) and torch.equal(qa.U, qb.U)
+    check_bytes(c.x, p["inv_s"], qa.Xq.cpu().numpy(), sf_atoms_to_rowmajor(qa.Xsf.cpu().numpy(), M, K),
+                float(qa.t_x.cpu()[0]))

@@ -212,6 +212,20 @@ def test_largest_block_takes_largest_scale_and_error_bound():
     assert np.all(err[np.broadcast_to(ok, err.shape)] <= 1.0 * np.broadcast_to(unit, err.shape)[np.broadcast_to(ok, err.shape)] * (1 + 1e-6))
 
 
+def test_row_subset_under_whole_tensor_scale():
+    """Once the tensor scale is fixed each row quantises on its own: a subset
+    of rows under the whole tensor's amax gives exactly those rows' bytes."""
+    g = rng(15)
+    x = bf16_round((g.standard_normal((40, 256)) * np.exp(g.standard_normal(256))).astype(np.float32))
+    inv_s = (1.0 / np.exp(0.2 * g.standard_normal(256))).astype(np.float32)
+    q, s, t, a = nvfp4.quantize_activation(x, inv_s)
+    rows = np.array([0, 7, 8, 39])
+    q2, s2, t2, a2 = nvfp4.quantize_activation(x, inv_s, rows)
+    assert t2 == t and a2 == a
+    np.testing.assert_array_equal(q2, q[rows])
+    np.testing.assert_array_equal(s2, s[rows])
+
+
 def test_all_zero_tensor():
     c, s, t, amax = nvfp4.quantize(np.zeros((4, 64), np.float32))
     assert amax == 0 and t == 1.0
