@@ -368,6 +368,59 @@ int w4a4_device_status(int* status, int reset) {
   return W4A4_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free activation quantisation.  Its scratch is this file-scope
+// device array; host code cannot use the symbol as a device address, so the
+// address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[w4a4::kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (set up on the
+// first call per device), or nullptr on failure.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= w4a4::kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" {
+
+int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx, const float* inv_s, const void* L1t,
+                               int r, const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U,
+                               void* stream) {
+  if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  const size_t need = nvfp4_quant_workspace_bytes(M, K, r);
+  if (need > W4A4_NOALLOC_SCRATCH_BYTES) return W4A4_ERR_SCRATCH_LIMIT;
+  if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;
+  if (r > 0 && (!L1t || !t_w || !U)) return W4A4_ERR_NULL;
+  DeviceInfo* dev = nullptr;
+  int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  void* scratch = noalloc_scratch();
+  if (scratch == nullptr) return W4A4_ERR_CUDA;
+  return nvfp4_quantize_act(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, scratch,
+                            W4A4_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 const char* w4a4_status_string(int status) {
   switch (status) {
     case W4A4_OK: return "ok";
@@ -379,6 +432,7 @@ const char* w4a4_status_string(int status) {
     case W4A4_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case W4A4_ERR_DEVICE_TIMEOUT: return "a device-side pipeline wait exceeded its bound";
     case W4A4_ERR_ARG: return "an enum argument is out of range";
+    case W4A4_ERR_SCRATCH_LIMIT: return "the problem needs more scratch than the built-in no-alloc array holds";
     default: return "unknown status";
   }
 }

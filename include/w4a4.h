@@ -74,7 +74,8 @@ typedef enum {
   W4A4_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than required */
   W4A4_ERR_CUDA = -6,           /* a CUDA call or kernel launch failed */
   W4A4_ERR_DEVICE_TIMEOUT = -7, /* sticky device status: a bounded wait gave up */
-  W4A4_ERR_ARG = -8             /* an enum argument is out of range */
+  W4A4_ERR_ARG = -8,            /* an enum argument is out of range */
+  W4A4_ERR_SCRATCH_LIMIT = -9   /* problem needs more than the built-in scratch (no-alloc entry) */
 } w4a4_status;
 
 enum { W4A4_EPI_NONE = 0, W4A4_EPI_GELU_TANH = 1 };
@@ -161,6 +162,41 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K,
                 const float* inv_s, const void* L1t, const void* L2t, int r,
                 const void* bias, int epilogue, void* Y,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_quantize_act_noalloc -- nvfp4_quantize_act for callers that cannot
+ * allocate device memory.  The paper has no counterpart to this entry point;
+ * it exists for hosts that hand a layer only its inputs and outputs: for
+ * example an inference-engine plugin interface with no workspace slot, or a
+ * serving runtime that plans every device buffer ahead of time and forbids
+ * allocation while requests are in flight (cudaMalloc can synchronise the
+ * device and fragment the planned memory).
+ *
+ * Arguments, layouts and results are those of nvfp4_quantize_act, without
+ * the workspace: the scratch this computation needs (per-CTA amax partial
+ * maxima, per-row-block counters and fp32 low-rank partial sums) lives in a
+ * file-scope device array of W4A4_NOALLOC_SCRATCH_BYTES (16 MiB) built into
+ * the library; every GPU that loads the library holds that array until the
+ * process exits.  The entry point allocates nothing (no cudaMalloc, cudaFree
+ * or allocating library call).
+ *
+ * - Sizes whose scratch need, nvfp4_quant_workspace_bytes(M, K, r), exceeds
+ *   W4A4_NOALLOC_SCRATCH_BYTES are rejected with W4A4_ERR_SCRATCH_LIMIT
+ *   before anything is enqueued (with r = 32 this admits roughly M up to
+ *   100k tokens).
+ * - The first call on a device looks up the device address of the array
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ * - All calls share the one array, which keeps the last call's contents.  The
+ *   kernels rewrite every scratch value they read and clear the counters at
+ *   the start of each call, so no clearing is needed between calls, but calls
+ *   that overlap on the GPU (for example on two streams without ordering
+ *   between them) race on the array and give wrong results.
+ */
+#define W4A4_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
+                               const float* inv_s, const void* L1t, int r, const float* t_w,
+                               uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* stream);
 
 /* Copies the sticky device status word of the current device into *status
  * (W4A4_OK or W4A4_ERR_DEVICE_TIMEOUT) and clears it if reset != 0.  This call
