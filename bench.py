@@ -55,9 +55,21 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def ncu_traffic(kernel_src: str, summary: str):
+GEMM_SOURCES = ["bit_diffusion_transformer_nvfp4_b200/csrc/gemm.cuh",
+                "bit_diffusion_transformer_nvfp4_b200/csrc/gemm2.cuh",
+                "bit_diffusion_transformer_nvfp4_b200/csrc/sm100.cuh"]
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel_srcs, summary: str):
     """DRAM bytes per launch from the committed ncu summary, if that summary
-    was taken on the current kernel source (hash match); else None."""
+    was taken on the current kernel sources (hash match); else None."""
     path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
@@ -66,7 +78,7 @@ def ncu_traffic(kernel_src: str, summary: str):
     h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", text)
     if not m or not h:
         return None
-    cur = hashlib.sha256(open(os.path.join(ROOT, kernel_src), "rb").read()).hexdigest()
+    cur = source_hash(kernel_srcs)
     if not cur.startswith(h.group(1)):
         return None
     return float(m.group(1))
@@ -251,7 +263,7 @@ def run_ours(args):
     gemm_avg_ms = statistics.mean(gemm_ms)
     g_fl = gemm_flops(M, K, N, r)
     achieved = g_fl / (gemm_avg_ms * 1e-3) / 1e12
-    traffic = ncu_traffic("bit_diffusion_transformer_nvfp4_b200/csrc/gemm.cuh", "gemm_flux1024_qkv_ncu.md")
+    traffic = ncu_traffic(GEMM_SOURCES, "gemm_flux1024_qkv_ncu.md")
     clocks = ClockSampler.summarise(clock_rows)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
@@ -263,7 +275,7 @@ def run_ours(args):
         "pct_fp4_peak": round(100.0 * value / (world * fp4_peak), 2),
         "fp4_peak_tflops": round(fp4_peak, 1),
         "fp4_peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOPS x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
-        "roofline": {"kernel": "gemm_kernel (block-scaled FP4 + low-rank + bias epilogue)", "bound": "tensor",
+        "roofline": {"kernel": "gemm2_kernel (CTA-pair block-scaled FP4 + low-rank + bias epilogue)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
                      "peak_kind": f"{peak_kind} (bf16 burst x4)", "launch_ms": round(gemm_avg_ms, 5),

@@ -1,0 +1,320 @@
+// gemm2.cuh -- the W4A4 GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same computation as gemm.cuh (block-scaled FP4 main product, hi|lo
+// low-rank pass into the same fp32 TMEM accumulator, bias / GELU / bf16
+// epilogue), restructured so that two SMs share one 256 x BN output tile:
+//
+//   * each CTA of the pair TMA-loads its own 128 rows of A (activation codes),
+//     its own half (BN/2 rows) of B (weight codes), its 128 rows' scale atoms
+//     and all BN rows' weight scale atoms; the loads of both CTAs complete on
+//     the even CTA's ring barrier;
+//   * the even CTA's MMA thread copies the scale atoms into both TMEMs and
+//     issues M=256 MMAs that read A and B from both CTAs' shared memory, so
+//     per SM the shared-memory traffic per FLOP is about half that of a
+//     single-CTA 128 x 256 tile;
+//   * ring stages and the accumulator are handed back with multicast
+//     tcgen05.commit to both CTAs; the odd CTA's epilogue releases the
+//     accumulator with remote mbarrier arrives;
+//   * the epilogue stages bf16 results in 64-byte-swizzled shared memory and
+//     writes them with TMA stores (full 64-byte rows, clipped at the edges).
+//
+// One persistent CTA pair per two SMs; 320 threads per CTA: warp 0 TMA
+// producer, warp 1 TMEM owner (+ MMA issuer in the even CTA), warps 2-9
+// epilogue.
+#pragma once
+
+#include "gemm.cuh"
+#include "sm100.cuh"
+
+namespace w4a4 {
+
+template <int BN_, int STAGES_>
+struct Gemm2Cfg {
+  static constexpr int BN = BN_;                       // tile width (output columns)
+  static constexpr int BH = BN / 2;                    // B rows held by each CTA
+  static constexpr int STAGES = STAGES_;
+  static constexpr int BM = 128;                       // rows per CTA (256 per pair)
+  static constexpr int BK = 256;
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BH * 128;
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_RB = BN / 128;              // 128-row scale blocks per tile
+  static constexpr int SFB_BYTES = SFB_RB * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int LR_BYTES = BM * 128 + BH * 64;  // U tile + this CTA's L2t half
+  static constexpr int SF_COLS = 16 + 4 * 2 * SFB_RB;
+  static constexpr int NUM_ACC = (2 * BN + SF_COLS <= 512) ? 2 : 1;
+  static constexpr int SFA_COL = NUM_ACC * BN;
+  static constexpr int SFB_COL = SFA_COL + 16;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int HALF = BN / 2;                  // columns per epilogue warp
+  static constexpr int EPI_BUF = 32 * 64;              // 32 rows x 32 bf16, one staging buffer
+  static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int SMEM = STAGE_BYTES * STAGES + EPI_BYTES + 1024 + 256;
+  static_assert(SFB_COL + 4 * 2 * SFB_RB <= TMEM_COLS, "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(BN % 128 == 0 && HALF % 32 == 0, "tile shape");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                 const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_l2,
+                 const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+  constexpr int BN = C::BN, STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* epi_smem = smem + C::STAGE_BYTES * STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + C::NUM_ACC;
+  uint64_t* drain = acc_empty + C::NUM_ACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const bool lr = p.has_lr != 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < C::NUM_ACC; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), 2 * C::EPI_WARPS);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_sfa);
+    tma_prefetch_desc(&tm_sfb);
+    tma_prefetch_desc(&tm_y);
+    if (lr) {
+      tma_prefetch_desc(&tm_u);
+      tma_prefetch_desc(&tm_l2);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int m_tiles = (p.M + 2 * C::BM - 1) / (2 * C::BM);
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int total = m_tiles * n_tiles;
+  const int nkb = p.K / C::BK;
+  const int pair = blockIdx.x >> 1;
+  const int pairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += pairs) {
+        const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+        const int n0 = (tile / m_tiles) * BN;
+        const int nb0 = n0 + static_cast<int>(rank) * C::BH;
+        if (lr) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* st = smem + s * C::STAGE_BYTES;
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * C::LR_BYTES);
+          tma_load_2d_pair(smem_u32(st), &tm_u, bar, 0, m0);
+          tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tm_l2, bar, 0, nb0);
+          ++it;
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* st = smem + s * C::STAGE_BYTES;
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(smem_u32(st), &tm_a, bar, kb * 128, m0);
+          tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tm_b, bar, kb * 128, nb0);
+          tma_load_3d_pair(smem_u32(st + C::A_BYTES + C::B_BYTES), &tm_sfa, bar, 0, kb * 4, m0 / 128);
+          tma_load_3d_pair(smem_u32(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES), &tm_sfb, bar, 0, kb * 4,
+                           n0 / 128);
+          ++it;
+        }
+      }
+      // The even CTA's ring barriers count both CTAs' bytes: there, wait
+      // (bounded) for the newest fills to land before shared memory goes away.
+      if (leader) {
+        const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0u;
+        for (uint32_t j = first; j < it; ++j) mbar_wait_drain(smem_u32(&full[j % STAGES]), (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      constexpr uint32_t kIdescF4 = idesc_nvf4(256, BN);
+      constexpr uint32_t kIdescBf = idesc_bf16(256, BN);
+      uint32_t it = 0, tcount = 0;
+      for (int tile = pair; tile < total; tile += pairs) {
+        const uint32_t acc = tcount % C::NUM_ACC;
+        const uint32_t aph = (tcount / C::NUM_ACC) & 1;
+        if (!mbar_wait(smem_u32(&acc_empty[acc]), aph ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        bool first = true;
+        bool ok = true;
+        if (lr) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, p.status)) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(b_base + 32 * (k & 1), 16, 512, kSwizzle64B);
+            mma_bf16_pair(d, ad, bd, kIdescBf, k > 0 ? 1u : 0u);
+          }
+          tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);
+          ++it;
+          first = false;
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t b_base = a_base + C::A_BYTES;
+          const uint32_t sfa_base = b_base + C::B_BYTES;
+          const uint32_t sfb_base = sfa_base + C::SFA_BYTES;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tc_cp_32x128b_x4_pair(tmem + C::SFA_COL + 4 * j, smem_desc(sfa_base + 512 * j, 0, 128, kSwizzleNone));
+#pragma unroll
+            for (int rb = 0; rb < C::SFB_RB; ++rb)
+              tc_cp_32x128b_x4_pair(tmem + C::SFB_COL + 4 * C::SFB_RB * j + 4 * rb,
+                                    smem_desc(sfb_base + 2048 * rb + 512 * j, 0, 128, kSwizzleNone));
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t ad = smem_desc(a_base + 32 * j, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(b_base + 32 * j, 16, 1024, kSwizzle128B);
+            mma_nvf4_pair(d, ad, bd, kIdescF4, tmem + C::SFA_COL + 4 * j, tmem + C::SFB_COL + 4 * C::SFB_RB * j,
+                          (!first || j > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);
+          ++it;
+          first = false;
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(smem_u32(&acc_full[acc]), 0x3);
+        ++tcount;
+      }
+      tc_commit_pair(smem_u32(drain));
+      mbar_wait_drain(smem_u32(drain), 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int q = warp & 3;               // TMEM lane quarter (rows 32q..32q+31 of this CTA)
+    const int h = ew >> 2;                // column half
+    const float alpha = __fmul_rn(__ldg(p.t_x), __ldg(p.t_w));
+    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    uint8_t* stage_buf = epi_smem + ew * 2 * C::EPI_BUF;
+    uint32_t tcount = 0, chunk = 0;
+    for (int tile = pair; tile < total; tile += pairs) {
+      const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+      const int n0 = (tile / m_tiles) * BN;
+      const uint32_t acc = tcount % C::NUM_ACC;
+      const uint32_t aph = (tcount / C::NUM_ACC) & 1;
+      if (!mbar_wait(smem_u32(&acc_full[acc]), aph, abort_flag, p.status)) break;
+      tc_fence_after();
+      uint32_t r[C::HALF];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + h * C::HALF;
+#pragma unroll
+      for (int c = 0; c < C::HALF / 32; ++c)
+        tmem_ld_32cols(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * acc);
+
+      const int row0 = m0 + q * 32;
+#pragma unroll
+      for (int c = 0; c < C::HALF / 32; ++c, ++chunk) {
+        const int n = n0 + h * C::HALF + 32 * c;
+        uint8_t* buf = stage_buf + (chunk & 1) * C::EPI_BUF;
+        if (chunk >= 2) {
+          // the TMA store that last used this buffer has finished reading it
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+        }
+        uint32_t packed[16];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float b[8];
+          if (p.bias != nullptr && n + 8 * g < p.N) {
+            const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8 * g));
+            b[0] = bf16_lo(bw.x); b[1] = bf16_hi(bw.x); b[2] = bf16_lo(bw.y); b[3] = bf16_hi(bw.y);
+            b[4] = bf16_lo(bw.z); b[5] = bf16_hi(bw.z); b[6] = bf16_lo(bw.w); b[7] = bf16_hi(bw.w);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) b[j] = 0.0f;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            float y0 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j])), b[j]);
+            float y1 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j + 1])), b[j + 1]);
+            if (p.epi == 1) {
+              y0 = gelu_tanh_f32(y0);
+              y1 = gelu_tanh_f32(y1);
+            }
+            packed[4 * g + j / 2] = pack_bf16x2(y0, y1);
+          }
+        }
+        // row `lane` of a 32 x 32 bf16 box, 64-byte rows, 64-byte swizzle
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int phys = g ^ ((lane >> 1) & 3);
+          *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
+              make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, smem_u32(buf), n, row0);
+          bulk_commit_group();
+        }
+      }
+      ++tcount;
+    }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its peer may still signal it or read its TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace w4a4

@@ -13,6 +13,7 @@
 
 #include "../../include/w4a4.h"
 #include "gemm.cuh"
+#include "gemm2.cuh"
 #include "quant.cuh"
 
 namespace w4a4 {
@@ -78,6 +79,11 @@ int device_setup(DeviceInfo** out) {
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G256>, cudaFuncAttributeMaxDynamicSharedMemorySize, G256::SMEM) ==
              cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G192>, cudaFuncAttributeMaxDynamicSharedMemorySize, G192::SMEM) ==
+             cudaSuccess;
+  using P256 = Gemm2Cfg<256, 5>;
+  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P256>, cudaFuncAttributeMaxDynamicSharedMemorySize, P256::SMEM) ==
+             cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P256>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) ==
              cudaSuccess;
   if (!attr_ok) { cudaGetLastError(); return W4A4_ERR_CUDA; }
   d.ok = true;
@@ -229,6 +235,68 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   return W4A4_OK;
 }
 
+// The CTA-pair kernel: 256 x BN tiles on two SMs (cluster of 2).
+template <class C>
+int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                     int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                     const void* bias, int epi, void* Y, int64_t ldy, cudaStream_t stream, DeviceInfo* dev) {
+  CUtensorMap ta, tb, tsa, tsb, tu, tl, ty;
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(K / 2), 128u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  if (!encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
+                 static_cast<uint64_t>(K / 2), 128u, static_cast<uint32_t>(C::BH), CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  if (!encode_sf(&tsa, Xsf, M, K, 1)) return W4A4_ERR_CUDA;
+  if (!encode_sf(&tsb, Wsf, N, K, static_cast<uint32_t>(C::SFB_RB))) return W4A4_ERR_CUDA;
+  if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(ldy) * 2, 32u, 32u, CU_TENSOR_MAP_SWIZZLE_64B))
+    return W4A4_ERR_CUDA;
+  if (r > 0) {
+    if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, 64u, static_cast<uint64_t>(M), 128u, 64u, 128u,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return W4A4_ERR_CUDA;
+    if (!encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2t, 32u, static_cast<uint64_t>(N), 64u, 32u,
+                   static_cast<uint32_t>(C::BH), CU_TENSOR_MAP_SWIZZLE_64B))
+      return W4A4_ERR_CUDA;
+  } else {
+    tu = ta;
+    tl = ta;
+  }
+  GemmParams p;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.ldy = ldy;
+  p.t_x = t_x;
+  p.t_w = t_w;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.has_lr = r > 0 ? 1 : 0;
+  p.epi = epi;
+  p.status = dev->status_ptr;
+  const int64_t tiles = ceil_div(M, 2 * C::BM) * ceil_div(N, C::BN);
+  const int64_t max_pairs = dev->num_sms / 2;
+  const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm2_kernel<C>, ta, tb, tsa, tsb, tu, tl, ty, p) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  return W4A4_OK;
+}
+
 int check_gemm_args(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                     int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
                     const void* bias, int epi, const void* Y, int64_t ldy) {
@@ -322,7 +390,11 @@ int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const voi
   if (st != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // 192-wide tiles (double-buffered accumulator) when N allows, else 256.
+  // CTA pairs (256 x 256 tiles) once there are at least two row blocks;
+  // single-CTA 128 x 192 / 128 x 256 tiles for a single row block.
+  if (M > 128)
+    return launch_gemm_pair<Gemm2Cfg<256, 5>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
+                                              s, dev);
   if (N % 192 == 0)
     return launch_gemm_cfg<GemmCfg<192, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
                                             s, dev);
