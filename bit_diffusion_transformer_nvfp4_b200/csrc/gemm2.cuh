@@ -38,7 +38,9 @@ struct Gemm2Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BH * 128;
   static constexpr int SFA_BYTES = 4 * 512;
-  static constexpr int SFB_RB = BN / 128;              // 128-row scale blocks per tile
+  // 128-row weight-scale blocks a tile can touch (a 192-wide tile may start
+  // 64 rows into a block)
+  static constexpr int SFB_RB = BN / 128 + (BN % 128 ? 1 : 0);
   static constexpr int SFB_BYTES = SFB_RB * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int LR_BYTES = BM * 128 + BH * 64;  // U tile + this CTA's L2t half
@@ -56,7 +58,7 @@ struct Gemm2Cfg {
   static_assert(SFB_COL + 4 * 2 * SFB_RB <= TMEM_COLS, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(BN % 128 == 0 && HALF % 32 == 0, "tile shape");
+  static_assert(BN % 64 == 0 && HALF % 32 == 0, "tile shape");
 };
 
 template <class C>
@@ -176,6 +178,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (!mbar_wait(smem_u32(&acc_empty[acc]), aph ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
+        // a tile starting 64 rows into a weight-scale block reads its scales
+        // two TMEM columns further on
+        const uint32_t sfb_shift = static_cast<uint32_t>(((tile / m_tiles) * BN % 128) / 32);
         bool first = true;
         bool ok = true;
         if (lr) {
@@ -216,7 +221,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int j = 0; j < 4; ++j) {
             const uint64_t ad = smem_desc(a_base + 32 * j, 16, 1024, kSwizzle128B);
             const uint64_t bd = smem_desc(b_base + 32 * j, 16, 1024, kSwizzle128B);
-            mma_nvf4_pair(d, ad, bd, kIdescF4, tmem + C::SFA_COL + 4 * j, tmem + C::SFB_COL + 4 * C::SFB_RB * j,
+            mma_nvf4_pair(d, ad, bd, kIdescF4, tmem + C::SFA_COL + 4 * j,
+                          tmem + C::SFB_COL + 4 * C::SFB_RB * j + sfb_shift,
                           (!first || j > 0) ? 1u : 0u);
           }
           tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);

@@ -44,6 +44,12 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ------------------------------------------------------------------ pass 1
+// A warp reads 32 consecutive 16-byte vectors of one row per work item (a
+// row segment), so the channel index of each lane needs no division; every
+// lane keeps kAmaxUnroll loads in flight.  Plain cached loads leave the
+// tensor in L2 for pass 2.
+constexpr int kAmaxUnroll = 8;
+
 template <typename SrcT>
 __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restrict__ X, int64_t M,
                                                             int64_t K, int64_t ld,
@@ -52,59 +58,60 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restri
                                                             int* __restrict__ tickets,
                                                             int n_tickets) {
   constexpr int EPV = 16 / sizeof(SrcT);  // elements per 16-byte vector
-  const int64_t vec_per_row = K / EPV;
-  const int64_t total = M * vec_per_row;
+  const int lane = threadIdx.x & 31;
+  const int segs = static_cast<int>(K / (32 * EPV));  // row segments (K % 256 == 0)
+  const int64_t items = M * segs;
+  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   float m = 0.0f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  auto absmax_vec = [&](int64_t i, const uint4 raw) {
-    const int64_t row = i / vec_per_row;
-    const int64_t col = (i - row * vec_per_row) * EPV;
-    float v[EPV];
-    if constexpr (sizeof(SrcT) == 2) {
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  for (int64_t base = warp_global * kAmaxUnroll; base < items; base += warps * kAmaxUnroll) {
+    uint4 raw[kAmaxUnroll];
+    int col[kAmaxUnroll];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[2 * j] = bf16_lo(w[j]);
-        v[2 * j + 1] = bf16_hi(w[j]);
-      }
-    } else {
-      v[0] = __uint_as_float(raw.x);
-      v[1] = __uint_as_float(raw.y);
-      v[2] = __uint_as_float(raw.z);
-      v[3] = __uint_as_float(raw.w);
-    }
-    if (inv_s != nullptr) {
-#pragma unroll
-      for (int j = 0; j < EPV; j += 4) {
-        const float4 s = __ldg(reinterpret_cast<const float4*>(inv_s + col + j));
-        v[j] = __fmul_rn(v[j], s.x);
-        v[j + 1] = __fmul_rn(v[j + 1], s.y);
-        v[j + 2] = __fmul_rn(v[j + 2], s.z);
-        v[j + 3] = __fmul_rn(v[j + 3], s.w);
+    for (int u = 0; u < kAmaxUnroll; ++u) {
+      const int64_t it = base + u;
+      col[u] = -1;
+      if (it < items) {
+        const int64_t row = it / segs;
+        const int seg = static_cast<int>(it - row * segs);
+        col[u] = (seg * 32 + lane) * EPV;
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(X + row * ld + col[u]));
       }
     }
 #pragma unroll
-    for (int j = 0; j < EPV; ++j) m = fmaxf(m, fabsf(v[j]));
-  };
-  auto load = [&](int64_t i) {
-    const int64_t row = i / vec_per_row;
-    const int64_t col = (i - row * vec_per_row) * EPV;
-    return __ldcs(reinterpret_cast<const uint4*>(X + row * ld + col));
-  };
-  int64_t i = i0;
-  // four independent 16-byte loads in flight per thread
-  for (; i + 3 * stride < total; i += 4 * stride) {
-    const uint4 a = load(i), b = load(i + stride), c = load(i + 2 * stride), d = load(i + 3 * stride);
-    absmax_vec(i, a);
-    absmax_vec(i + stride, b);
-    absmax_vec(i + 2 * stride, c);
-    absmax_vec(i + 3 * stride, d);
+    for (int u = 0; u < kAmaxUnroll; ++u) {
+      if (col[u] < 0) continue;
+      float v[EPV];
+      if constexpr (sizeof(SrcT) == 2) {
+        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[2 * j] = bf16_lo(w[j]);
+          v[2 * j + 1] = bf16_hi(w[j]);
+        }
+      } else {
+        v[0] = __uint_as_float(raw[u].x);
+        v[1] = __uint_as_float(raw[u].y);
+        v[2] = __uint_as_float(raw[u].z);
+        v[3] = __uint_as_float(raw[u].w);
+      }
+      if (inv_s != nullptr) {
+#pragma unroll
+        for (int j = 0; j < EPV; j += 4) {
+          const float4 s = __ldg(reinterpret_cast<const float4*>(inv_s + col[u] + j));
+          v[j] = __fmul_rn(v[j], s.x);
+          v[j + 1] = __fmul_rn(v[j + 1], s.y);
+          v[j + 2] = __fmul_rn(v[j + 2], s.z);
+          v[j + 3] = __fmul_rn(v[j + 3], s.w);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < EPV; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
   }
-  for (; i < total; i += stride) absmax_vec(i, load(i));
   __shared__ float red[kAmaxThreads / 32];
   m = warp_max(m);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x < 32) {
     float v = threadIdx.x < kAmaxThreads / 32 ? red[threadIdx.x] : 0.0f;
@@ -131,6 +138,7 @@ struct QuantParams {
   int* tickets;            // [row_blocks]
   int chunks_per_split;
   int splits;
+  int row_blocks;
   int has_lr;
   int* status;
 };
@@ -176,6 +184,58 @@ __device__ __forceinline__ float tensor_scale_from(float amax) {
   float t = __fdiv_rn(amax, 2688.0f);
   if (!(t >= 1.17549435e-38f)) t = 1.0f;  // not a normal number -> 1
   return t;
+}
+
+// The last K slice of a row block sums the fp32 partials in slice order,
+// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row.
+__device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, int64_t rows_pad, int64_t prow,
+                                                 int64_t row) {
+  __threadfence();
+  float acc[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+  for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
+    // the loads of two slices are in flight together; the sums still run in
+    // slice order
+    float4 w[2][8];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (sp0 + q < p.splits) {
+        const float4* src =
+            reinterpret_cast<const float4*>(p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow) * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[q][j] = __ldcg(src + j);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (sp0 + q < p.splits) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc[4 * j] = __fadd_rn(acc[4 * j], w[q][j].x);
+          acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], w[q][j].y);
+          acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], w[q][j].z);
+          acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], w[q][j].w);
+        }
+      }
+    }
+  }
+  if (row < p.M) {
+    const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
+      const uint32_t h = pack_bf16x2(a0, a1);
+      hi[j / 2] = h;
+      lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
+    }
+    uint4* dst2 = reinterpret_cast<uint4*>(p.u_out + row * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst2[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst2[4 + j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+  }
 }
 
 template <typename SrcT>
@@ -300,7 +360,6 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
       if (!mbar_wait(smem_u32(&full[s]), (i / S) & 1, abort_flag, p.status)) break;
       const uint8_t* tile = smem + s * Tile::kStageBytes;
       const int kc = kc0 + i;
-      const int k0 = kc * kQChunk;
 
       float x[64];
 #pragma unroll
@@ -423,54 +482,406 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
   }
   __syncthreads();
   if (*last_flag && warp < kQComputeWarps) {
-    // the last K slice of this row block sums the partials in slice order
-    __threadfence();
     const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-    float acc[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
-    for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
-      // the loads of two slices are in flight together; the sums still run
-      // in slice order
-      float4 w[2][8];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (sp0 + q < p.splits) {
-          const float4* src =
-              reinterpret_cast<const float4*>(p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow) * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) w[q][j] = __ldcg(src + j);
+    finalize_lowrank(p, t, rows_pad, prow, row);
+  }
+}
+
+// ------------------------------------------------------------------ fused single pass
+// When every (128-row block, K slice) tile of the activation fits in the
+// shared memory of one co-resident wave of CTAs (one CTA per SM, up to
+// kFusedMaxChunks 64-wide chunks each), the activation is read from HBM once:
+// each CTA TMA-loads all of its chunks and keeps them resident, reduces its
+// partial amax, meets every other CTA at a grid barrier (cooperative launch,
+// bounded spin), then quantises from shared memory.  The U = X L1 MMAs run as
+// the chunks land (L1t streams through a small ring).
+constexpr int kFusedMaxChunks = 12;
+constexpr int kFusedL1Ring = 7;  // L1t tiles in flight: as many as fit beside the resident X
+
+struct FusedQuantSmem {
+  static constexpr int kXBytes = kFusedMaxChunks * kQRows * kQChunk * 2;   // 192 KB
+  static constexpr int kL1Bytes = kFusedL1Ring * 32 * kQChunk * 2;         // 28 KB
+  static constexpr int kInvBytes = kFusedMaxChunks * kQChunk * 4;          // 3 KB
+  static constexpr int kRqBytes = 256 * 4;                                 // 1/(dec(e) t) per scale code
+  static constexpr int kBarBytes = 512;
+  static constexpr int kBytes = kXBytes + kL1Bytes + kInvBytes + kRqBytes + kBarBytes + 1024;
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+// Fused kernel roles (16 warps).  Warps 0-11 compute in three groups of four:
+// group g owns chunks g, g+3, g+6, g+9 of the slice and thread (g, r) row r of
+// each.  Warp 12 is the TMA producer and warp 13 the TMEM owner and U-MMA
+// issuer; after that, warps 12-15 (one per TMEM lane quarter) move the partial
+// U out of TMEM and, once every slice of the row block has its partial out
+// (a per-row-block ticket), sum the partials of this CTA's share of the rows.
+// The compute warps never wait for them.
+constexpr int kFGroups = 3;
+constexpr int kFComputeWarps = 4 * kFGroups;
+constexpr int kFChunksPerThread = kFusedMaxChunks / kFGroups;
+constexpr int kFProducerWarp = 12;
+constexpr int kFMmaWarp = 13;
+constexpr int kFUWarp0 = 12;  // warps 12-15 cover TMEM lane quarters 0-3
+constexpr int kFThreads = 32 * 16;
+static_assert(kFusedMaxChunks % kFGroups == 0, "chunk groups");
+static_assert(kFComputeWarps * 32 >= 256, "one thread per scale code fills the multiplier table");
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+static_assert(kFUWarp0 % 4 == 0 && kFThreads == 32 * (kFUWarp0 + 4), "lane quarters");
+
+// Blackwell packed fp32 multiply: two IEEE round-to-nearest products.
+__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Bounded spin until a global counter reaches ``target``; false on timeout
+// (then the abort flag and the device status are set).
+__device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target, volatile int* abort, int* status) {
+  const long long start = clock64();
+  while (ld_acquire_gpu(ctr) < target) {
+    if (*abort) return false;
+    if (clock64() - start > kWaitBoundCycles) {
+      *abort = 1;
+      if (status) atomicExch(status, kStatusTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+// Eight smoothed values of row ``r``, 16-byte unit ``u`` (elements 8u..8u+7)
+// of a resident bf16 chunk.
+__device__ __forceinline__ void load_unit(const uint8_t* tile, const float* inv, bool has_inv, int r, int u,
+                                          float (&v)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(tile + r * 128 + ((u ^ (r & 7)) << 4));
+  v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x);
+  v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+  v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z);
+  v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+  if (has_inv) {
+    const float4 s0 = reinterpret_cast<const float4*>(inv)[2 * u];
+    const float4 s1 = reinterpret_cast<const float4*>(inv)[2 * u + 1];
+    mul2_rn(v[0], v[1], v[0], v[1], s0.x, s0.y);
+    mul2_rn(v[2], v[3], v[2], v[3], s0.z, s0.w);
+    mul2_rn(v[4], v[5], v[4], v[5], s1.x, s1.y);
+    mul2_rn(v[6], v[7], v[6], v[7], s1.z, s1.w);
+  }
+}
+
+__global__ void __launch_bounds__(kFThreads, 1)
+    quant_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
+                       const QuantParams p, unsigned* grid_sync) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = smem;
+  uint8_t* l1s = smem + FusedQuantSmem::kXBytes;
+  float* invs = reinterpret_cast<float*>(l1s + FusedQuantSmem::kL1Bytes);
+  float* rq_tab = invs + kFusedMaxChunks * kQChunk;
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(rq_tab) + FusedQuantSmem::kRqBytes);
+  uint64_t* l1_full = full + kFusedMaxChunks;
+  uint64_t* l1_empty = l1_full + kFusedL1Ring;
+  uint64_t* drain = l1_empty + kFusedL1Ring;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);  // kFComputeWarps floats
+  float* t_shared = reinterpret_cast<float*>(tmem_slot + 2 + kFComputeWarps);
+  unsigned* counter = grid_sync;       // CTAs that have contributed
+  unsigned* amax_bits = grid_sync + 1; // running max of the CTA maxima (non-negative floats order as bits)
+  unsigned* tickets = grid_sync + 2;   // per row block: slices whose partial U is out
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int rb = blockIdx.x / p.splits;
+  const int split = blockIdx.x % p.splits;
+  const int chunks = static_cast<int>(p.K / kQChunk);
+  const int kc0 = split * p.chunks_per_split;
+  const int kc1 = min(kc0 + p.chunks_per_split, chunks);
+  const int n = kc1 - kc0;
+  const bool lr = p.has_lr != 0;
+  const bool has_inv = p.inv_s != nullptr;
+  const int64_t rows_pad = static_cast<int64_t>(p.row_blocks) * kQRows;
+
+  if (tid == 0) {
+    for (int c = 0; c < kFusedMaxChunks; ++c) mbar_init(smem_u32(&full[c]), 1);
+    for (int r = 0; r < kFusedL1Ring; ++r) {
+      mbar_init(smem_u32(&l1_full[r]), 1);
+      mbar_init(smem_u32(&l1_empty[r]), 1);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (lr && warp == kFMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = lr ? *tmem_slot : 0u;
+
+  float bmax[4 * kFChunksPerThread];  // compute threads: block maxima of their row
+  const int r = tid & (kQRows - 1);
+  const int grp = warp >> 2;
+
+  if (warp >= kFUWarp0) {
+    if (warp == kFProducerWarp && lane == 0) {
+      // ---------------------------------------------------- all loads up front
+      // Each chunk's L1t tile is queued right behind its X tile (while ring
+      // slots last), so the U MMAs follow the chunks as they land; the
+      // remaining L1t tiles reuse slots as the MMAs free them.
+      tma_prefetch_desc(&tm_x);
+      if (lr) tma_prefetch_desc(&tm_l1);
+      auto load_l1 = [&](int c) {
+        const int s = c % kFusedL1Ring;
+        const uint32_t bar = smem_u32(&l1_full[s]);
+        mbar_arrive_expect_tx(bar, 32 * kQChunk * 2);
+        tma_load_2d(smem_u32(l1s + s * 32 * kQChunk * 2), &tm_l1, bar, (kc0 + c) * kQChunk, 0);
+      };
+      for (int c = 0; c < n; ++c) {
+        const int kx = (kc0 + c) * kQChunk;
+        const uint32_t bar = smem_u32(&full[c]);
+        const uint32_t inv_bytes = has_inv ? kQChunk * 4 : 0;
+        mbar_arrive_expect_tx(bar, kQRows * kQChunk * 2 + inv_bytes);
+        tma_load_2d(smem_u32(xs + c * kQRows * kQChunk * 2), &tm_x, bar, kx, rb * kQRows);
+        if (inv_bytes) bulk_load(smem_u32(invs + c * kQChunk), p.inv_s + kx, inv_bytes, bar);
+        if (lr && c < kFusedL1Ring) load_l1(c);
+      }
+      if (lr) {
+        for (int c = kFusedL1Ring; c < n; ++c) {
+          const int s = c % kFusedL1Ring;
+          if (!mbar_wait(smem_u32(&l1_empty[s]), ((c / kFusedL1Ring) - 1) & 1, abort_flag, p.status)) break;
+          load_l1(c);
         }
       }
+    } else if (warp == kFMmaWarp && lane == 0 && lr) {
+      // ---------------------------------------------------- U = X L1 as the chunks land
+      for (int c = 0; c < n; ++c) {
+        const int s = c % kFusedL1Ring;
+        if (!mbar_wait(smem_u32(&full[c]), 0, abort_flag, p.status)) break;
+        if (!mbar_wait(smem_u32(&l1_full[s]), (c / kFusedL1Ring) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(xs + c * kQRows * kQChunk * 2);
+        const uint32_t b_base = smem_u32(l1s + s * 32 * kQChunk * 2);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (sp0 + q < p.splits) {
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
+          mma_bf16(tmem, ad, bd, idesc_bf16(128, 32), (c > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&l1_empty[s]));
+      }
+      tc_commit(smem_u32(drain));
+    }
+    __syncwarp();
+    if (lr) {
+      // ------------------------------------------------------ partial U out of TMEM
+      const int quarter = warp - kFUWarp0;
+      uint32_t u[32];
+      const bool ok = mbar_wait(smem_u32(drain), 0, abort_flag, p.status);
+      __syncwarp();
+      tc_fence_after();
+      tmem_ld_32cols(tmem + (static_cast<uint32_t>(quarter * 32) << 16), u);
+      tmem_ld_wait();
+      if (!ok || n == 0) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            acc[4 * j] = __fadd_rn(acc[4 * j], w[q][j].x);
-            acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], w[q][j].y);
-            acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], w[q][j].z);
-            acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], w[q][j].w);
+        for (int j = 0; j < 32; ++j) u[j] = 0u;
+      }
+      const int64_t prow = static_cast<int64_t>(rb) * kQRows + quarter * 32 + lane;
+      float4* dst = reinterpret_cast<float4*>(p.u_part + (static_cast<int64_t>(split) * rows_pad + prow) * 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        dst[j] = make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
+                             __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
+      __threadfence();
+      tc_fence_before();
+      named_bar_sync(3, 128);  // the four U warps: TMEM read, partial out
+      if (warp == kFMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 32);
+      }
+      if (tid == 32 * kFUWarp0) red_release_add(tickets + rb, 1u);
+      // ---------------------------------------------------- wait for the tensor scale
+      named_bar_sync(2, kFThreads);
+      if (!*abort_flag) {
+        if (tid == 32 * kFUWarp0) spin_until(tickets + rb, static_cast<unsigned>(p.splits), abort_flag, p.status);
+        named_bar_sync(3, 128);
+        if (!*abort_flag) {
+          // -------------------------------------------------- this CTA's share of the U rows
+          // The slices of a row block split its 128 rows; four threads per
+          // row, eight columns each; the sum runs in slice order.
+          const float t = *t_shared;
+          const int ut = tid - 32 * kFUWarp0;
+          const int cg = ut & 3;
+          const int rows_per = (kQRows + p.splits - 1) / p.splits;
+          const int r_end = min(kQRows, (split + 1) * rows_per);
+          const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
+          for (int rr = split * rows_per + (ut >> 2); rr < r_end; rr += 32) {
+            const int64_t prow2 = static_cast<int64_t>(rb) * kQRows + rr;
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
+              float4 w[4][2];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (sp0 + q < p.splits) {
+                  const float4* src = reinterpret_cast<const float4*>(
+                      p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow2) * 32 + cg * 8);
+                  w[q][0] = __ldcg(src);
+                  w[q][1] = __ldcg(src + 1);
+                }
+              }
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (sp0 + q < p.splits) {
+#pragma unroll
+                  for (int hh = 0; hh < 2; ++hh) {
+                    acc[4 * hh] = __fadd_rn(acc[4 * hh], w[q][hh].x);
+                    acc[4 * hh + 1] = __fadd_rn(acc[4 * hh + 1], w[q][hh].y);
+                    acc[4 * hh + 2] = __fadd_rn(acc[4 * hh + 2], w[q][hh].z);
+                    acc[4 * hh + 3] = __fadd_rn(acc[4 * hh + 3], w[q][hh].w);
+                  }
+                }
+              }
+            }
+            if (prow2 < p.M) {
+              uint32_t hi[4], lo[4];
+#pragma unroll
+              for (int j = 0; j < 8; j += 2) {
+                const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
+                const uint32_t hb = pack_bf16x2(a0, a1);
+                hi[j / 2] = hb;
+                lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(hb)), __fsub_rn(a1, bf16_hi(hb)));
+              }
+              __nv_bfloat16* urow = p.u_out + prow2 * 64;
+              *reinterpret_cast<uint4*>(urow + cg * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+              *reinterpret_cast<uint4*>(urow + 32 + cg * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
           }
         }
       }
     }
-    if (row < p.M) {
-      const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
-      uint32_t hi[16], lo[16];
+  } else {
+    // ------------------------------------------------------ phase A: block maxima
+    float m = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
-        const uint32_t h = pack_bf16x2(a0, a1);
-        hi[j / 2] = h;
-        lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
+    for (int i = 0; i < kFChunksPerThread; ++i) {
+      const int c = grp + kFGroups * i;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) bmax[4 * i + b] = 0.0f;
+      if (c < n && mbar_wait(smem_u32(&full[c]), 0, abort_flag, p.status)) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float v[8];
+          load_unit(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, u, v);
+          float bm = bmax[4 * i + u / 2];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) bm = fmaxf(bm, fabsf(v[j]));
+          bmax[4 * i + u / 2] = bm;
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b) m = fmaxf(m, bmax[4 * i + b]);
       }
-      uint4* dst2 = reinterpret_cast<uint4*>(p.u_out + row * 64);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst2[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst2[4 + j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
     }
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+
+    // ------------------------------------------------------ grid barrier (compute warps)
+    named_bar_sync(1, 32 * kFComputeWarps);
+    if (tid == 0) {
+      float a = red[0];
+#pragma unroll
+      for (int w = 1; w < kFComputeWarps; ++w) a = fmaxf(a, red[w]);
+      atomicMax(amax_bits, __float_as_uint(a));
+      red_release_add(counter, 1u);
+      spin_until(counter, gridDim.x, abort_flag, p.status);
+      const float t = tensor_scale_from(__uint_as_float(ld_acquire_gpu(amax_bits)));
+      *t_shared = t;
+      if (blockIdx.x == 0) *p.t_out = t;
+    }
+    named_bar_sync(1, 32 * kFComputeWarps);
+    if (lr) named_bar_arrive(2, kFThreads);  // the tensor scale is out for the U warps
+    const float t = *t_shared;
+    if (*abort_flag) return;
+
+    // ------------------------------------------------------ phase B: scales and codes
+    // The code multiplier 1/(dec(e) t) of every scale code, once per CTA.
+    if (tid < 256) rq_tab[tid] = __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(tid)).y, t));
+    named_bar_sync(1, 32 * kFComputeWarps);
+    const float rt = __frcp_rn(t);
+    const int64_t row = static_cast<int64_t>(rb) * kQRows + r;
+    const bool row_ok = row < p.M;
+    const int64_t kbytes = p.K / 2;
+#pragma unroll
+    for (int i = 0; i < kFChunksPerThread; ++i) {
+      const int c = grp + kFGroups * i;
+      if (c < n) {
+        const int kc = kc0 + c;
+        uint32_t e4 = 0u;
+        uint32_t cw[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // two blocks' scale bytes in one conversion; byte 0 = block 2h
+          const uint32_t e2 = cvt_e4m3x2(__fdiv_rn(__fmul_rn(bmax[4 * i + 2 * h + 1], rt), 6.0f),
+                                         __fdiv_rn(__fmul_rn(bmax[4 * i + 2 * h], rt), 6.0f)) & 0xFFFFu;
+          e4 |= e2 << (16 * h);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int b = 2 * h + q;
+            const uint32_t e = (e2 >> (8 * q)) & 0xFFu;
+            cw[2 * b] = cw[2 * b + 1] = 0u;
+            if (e != 0u) {  // a zero scale leaves the block's codes +0
+              const float rq = rq_tab[e];
+#pragma unroll
+              for (int uu = 0; uu < 2; ++uu) {
+                float v[8];
+                load_unit(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
+                mul2_rn(v[0], v[1], v[0], v[1], rq, rq);
+                mul2_rn(v[2], v[3], v[2], v[3], rq, rq);
+                mul2_rn(v[4], v[5], v[4], v[5], rq, rq);
+                mul2_rn(v[6], v[7], v[6], v[7], rq, rq);
+                cw[2 * b + uu] = cvt_e2m1x8(v);
+              }
+            }
+          }
+        }
+        if (row_ok) {
+          uint4* dq = reinterpret_cast<uint4*>(p.q + row * kbytes + static_cast<int64_t>(kc) * 32);
+          dq[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          dq[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        }
+        const int64_t atom = static_cast<int64_t>(rb) * chunks + kc;
+        *reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (r & 31) * 16 + (r >> 5) * 4) = e4;
+      }
+    }
+  }
+  if (warp == kFProducerWarp && lane == 0) {
+    // no copy may still be landing when the CTA exits
+    for (int c = 0; c < n; ++c) mbar_wait_drain(smem_u32(&full[c]), 0);
   }
 }
 

@@ -14,6 +14,7 @@
 #include "../../include/w4a4.h"
 #include "gemm.cuh"
 #include "gemm2.cuh"
+
 #include "quant.cuh"
 
 namespace w4a4 {
@@ -74,6 +75,8 @@ int device_setup(DeviceInfo** out) {
                                   QuantTile<__nv_bfloat16>::kSmem) == cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(quant_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   QuantTile<float>::kSmem) == cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(quant_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FusedQuantSmem::kBytes) == cudaSuccess;
   using G256 = GemmCfg<256, 4>;
   using G192 = GemmCfg<192, 4>;
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G256>, cudaFuncAttributeMaxDynamicSharedMemorySize, G256::SMEM) ==
@@ -81,10 +84,12 @@ int device_setup(DeviceInfo** out) {
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G192>, cudaFuncAttributeMaxDynamicSharedMemorySize, G192::SMEM) ==
              cudaSuccess;
   using P256 = Gemm2Cfg<256, 5>;
+  using P192 = Gemm2Cfg<192, 5>;
   attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P256>, cudaFuncAttributeMaxDynamicSharedMemorySize, P256::SMEM) ==
              cudaSuccess;
-  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P256>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) ==
+  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P192>, cudaFuncAttributeMaxDynamicSharedMemorySize, P192::SMEM) ==
              cudaSuccess;
+
   if (!attr_ok) { cudaGetLastError(); return W4A4_ERR_CUDA; }
   d.ok = true;
   *out = &d;
@@ -129,7 +134,9 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
   q.splits = static_cast<int>(ceil_div(q.chunks, q.chunks_per_split));
   q.off_partials = 0;
   q.off_tickets = round256(sizeof(float) * kAmaxMaxBlocks);
-  q.off_upart = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks > 0 ? q.row_blocks : 1));
+  // per-row-block tickets, then the single-pass path's grid-barrier counter
+  // and tensor-amax word
+  q.off_upart = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks + 2));
   const size_t upart = r > 0 ? sizeof(float) * static_cast<size_t>(q.splits) * q.row_blocks * kQRows * 32 : 0;
   q.bytes = q.off_upart + round256(upart);
   return q;
@@ -137,10 +144,85 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
 
 bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0 && K <= (int64_t(1) << 30); }
 
+// Single-pass activation quantisation: every (row block, K slice) tile must
+// be resident at once, one CTA per SM.  Returns W4A4_OK, or -1 when the shape
+// or the device does not allow it (the caller then runs the two-pass path).
+int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld, const float* inv_s,
+                       const void* L1t, int r, const float* t_w, uint8_t* q, uint8_t* sf, float* t_out, void* U,
+                       void* ws, cudaStream_t stream, DeviceInfo* dev) {
+  const QuantPlan plan = quant_plan(M, K, r);
+  const int64_t rb = plan.row_blocks;
+  const int chunks = plan.chunks;
+  if (rb < 1 || rb > dev->num_sms) return -1;
+  int64_t want = ceil_div(chunks, kFusedMaxChunks);
+  const int64_t more = dev->num_sms / rb;
+  if (more > want) want = more;
+  if (want > chunks) want = chunks;
+  const int cps = static_cast<int>(ceil_div(chunks, want));
+  const int splits = static_cast<int>(ceil_div(chunks, cps));
+  if (cps > kFusedMaxChunks || rb * splits > dev->num_sms || splits > plan.splits) return -1;
+
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  // grid-barrier counter, tensor-amax bits, one ticket per row block
+  unsigned* grid_sync = reinterpret_cast<unsigned*>(w + plan.off_tickets);
+  if (cudaMemsetAsync(grid_sync, 0, sizeof(unsigned) * static_cast<size_t>(rb + 2), stream) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  CUtensorMap tm_x, tm_l1;
+  if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(ld) * 2, 64u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  if (r > 0) {
+    if (!encode_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, static_cast<uint64_t>(K), static_cast<uint64_t>(r),
+                   static_cast<uint64_t>(K) * 2, 64u, static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B))
+      return W4A4_ERR_CUDA;
+  } else {
+    tm_l1 = tm_x;
+  }
+  QuantParams p;
+  p.M = M;
+  p.K = K;
+  p.inv_s = inv_s;
+  p.partials = reinterpret_cast<float*>(w + plan.off_partials);
+  p.n_partials = static_cast<int>(rb * splits);
+  p.t_w = t_w;
+  p.q = q;
+  p.sf = sf;
+  p.t_out = t_out;
+  p.u_part = reinterpret_cast<float*>(w + plan.off_upart);
+  p.u_out = static_cast<__nv_bfloat16*>(U);
+  p.tickets = nullptr;
+  p.chunks_per_split = cps;
+  p.splits = splits;
+  p.row_blocks = static_cast<int>(rb);
+  p.has_lr = r > 0 ? 1 : 0;
+  p.status = dev->status_ptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rb * splits), 1, 1);
+  cfg.blockDim = dim3(kFThreads, 1, 1);
+  cfg.dynamicSmemBytes = FusedQuantSmem::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, p, grid_sync) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;  // not co-resident on this device: fall back
+  }
+  return W4A4_OK;
+}
+
 template <typename SrcT>
 int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* inv_s, const void* L1t, int r,
                  const float* t_w, uint8_t* q, uint8_t* sf, float* t_out, void* U, void* ws,
                  cudaStream_t stream, DeviceInfo* dev) {
+  if constexpr (sizeof(SrcT) == 2) {
+    const int st = launch_quant_fused(X, M, K, ld, inv_s, L1t, r, t_w, q, sf, t_out, U, ws, stream, dev);
+    if (st != -1) return st;
+  }
   const QuantPlan plan = quant_plan(M, K, r);
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* partials = reinterpret_cast<float*>(w + plan.off_partials);
@@ -148,8 +230,8 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   float* upart = reinterpret_cast<float*>(w + plan.off_upart);
 
   constexpr int EPV = 16 / sizeof(SrcT);
-  const int64_t vecs = M * (K / EPV);
-  int64_t grid1 = ceil_div(vecs, kAmaxThreads * 4);
+  const int64_t items = M * (K / (32 * EPV));  // warp work items (row segments)
+  int64_t grid1 = ceil_div(items, (kAmaxThreads / 32) * kAmaxUnroll);
   if (grid1 > kAmaxMaxBlocks) grid1 = kAmaxMaxBlocks;
   if (grid1 < 1) grid1 = 1;
   amax_kernel<SrcT><<<static_cast<unsigned>(grid1), kAmaxThreads, 0, stream>>>(
@@ -184,6 +266,7 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   p.tickets = tickets;
   p.chunks_per_split = plan.chunks_per_split;
   p.splits = plan.splits;
+  p.row_blocks = static_cast<int>(plan.row_blocks);
   p.has_lr = r > 0 ? 1 : 0;
   p.status = dev->status_ptr;
   const dim3 grid2(static_cast<unsigned>(plan.row_blocks), static_cast<unsigned>(plan.splits));
@@ -235,7 +318,7 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   return W4A4_OK;
 }
 
-// The CTA-pair kernel: 256 x BN tiles on two SMs (cluster of 2).
+// The CTA-pair kernels: 256 x BN tiles on two SMs (cluster of 2).
 template <class C>
 int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                      int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
