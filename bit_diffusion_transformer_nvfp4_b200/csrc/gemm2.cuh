@@ -8,19 +8,26 @@
 //     its own half (BN/2 rows) of B (weight codes), its 128 rows' scale atoms
 //     and all BN rows' weight scale atoms; the loads of both CTAs complete on
 //     the even CTA's ring barrier;
-//   * the even CTA's MMA thread copies the scale atoms into both TMEMs and
-//     issues M=256 MMAs that read A and B from both CTAs' shared memory, so
-//     per SM the shared-memory traffic per FLOP is about half that of a
-//     single-CTA 128 x 256 tile;
+//   * the even CTA's MMA thread issues M=256 MMAs that read A and B from both
+//     CTAs' shared memory, so per SM the shared-memory traffic per FLOP is
+//     about half that of a single-CTA 128 x 256 tile;
+//   * block scales bypass the tensor pipe: tcgen05.cp copies execute in the
+//     same in-order queue as the MMAs (twelve per 256-deep K step cost about
+//     as much as the four MMAs), so instead each CTA's scale atoms travel
+//     through their own small shared-memory ring, loaded several K steps
+//     ahead, and four scale warps per CTA (one per TMEM lane quarter) write
+//     them into a ring of TMEM scale slots with tcgen05.st; the MMA thread
+//     waits for a slot's eight warp arrivals and frees it with a multicast
+//     commit;
 //   * ring stages and the accumulator are handed back with multicast
 //     tcgen05.commit to both CTAs; the odd CTA's epilogue releases the
 //     accumulator with remote mbarrier arrives;
 //   * the epilogue stages bf16 results in 64-byte-swizzled shared memory and
 //     writes them with TMA stores (full 64-byte rows, clipped at the edges).
 //
-// One persistent CTA pair per two SMs; 320 threads per CTA: warp 0 TMA
+// One persistent CTA pair per two SMs; 448 threads per CTA: warp 0 TMA
 // producer, warp 1 TMEM owner (+ MMA issuer in the even CTA), warps 2-9
-// epilogue.
+// epilogue, warps 10-13 scale warps.
 #pragma once
 
 #include "gemm.cuh"
@@ -37,26 +44,34 @@ struct Gemm2Cfg {
   static constexpr int BK = 256;
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BH * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int LR_BYTES = BM * 128 + BH * 64;  // U tile + this CTA's L2t half
+  // scale ring: one slot per 256-deep K step, this CTA's 128 rows of A
+  // scales (4 atoms) and the weight scales of every 128-row block the tile
+  // touches (a 192-wide tile may start 64 rows into a block)
   static constexpr int SFA_BYTES = 4 * 512;
-  // 128-row weight-scale blocks a tile can touch (a 192-wide tile may start
-  // 64 rows into a block)
   static constexpr int SFB_RB = BN / 128 + (BN % 128 ? 1 : 0);
   static constexpr int SFB_BYTES = SFB_RB * 4 * 512;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int LR_BYTES = BM * 128 + BH * 64;  // U tile + this CTA's L2t half
-  static constexpr int SF_COLS = 16 + 4 * 2 * SFB_RB;
-  static constexpr int NUM_ACC = (2 * BN + SF_COLS <= 512) ? 2 : 1;
-  static constexpr int SFA_COL = NUM_ACC * BN;
-  static constexpr int SFB_COL = SFA_COL + 16;
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int SF_STAGES = 5;
+  // TMEM: accumulator(s), then scale slots of SF_COLS columns (per K-block j
+  // of the step: A scales at 4j, weight-scale block rb at 16 + 4*SFB_RB*j + 4*rb)
+  static constexpr int SF_COLS = 16 + 4 * 4 * SFB_RB;
+  static constexpr int NUM_ACC = (2 * BN + 2 * SF_COLS <= 512) ? 2 : 1;
+  static constexpr int SF_COL0 = NUM_ACC * BN;
+  static constexpr int NB_TSF_FIT = (512 - SF_COL0) / SF_COLS;
+  static constexpr int NB_TSF = NB_TSF_FIT < 6 ? NB_TSF_FIT : 6;
   static constexpr int TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int SF_WARP0 = 2 + EPI_WARPS;       // warps 10-13
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * 4;
   static constexpr int HALF = BN / 2;                  // columns per epilogue warp
   static constexpr int EPI_BUF = 32 * 64;              // 32 rows x 32 bf16, one staging buffer
   static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
-  static constexpr int SMEM = STAGE_BYTES * STAGES + EPI_BYTES + 1024 + 256;
-  static_assert(SFB_COL + 4 * 2 * SFB_RB <= TMEM_COLS, "TMEM budget");
-  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static constexpr int SMEM = STAGE_BYTES * STAGES + SF_STAGE_BYTES * SF_STAGES + EPI_BYTES + 1024 + 512;
+  static_assert(NB_TSF >= 2 && SF_COL0 + NB_TSF * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COLS % 16 == 0, "scale slot written 16 columns at a time");
+  static_assert(STAGE_BYTES % 1024 == 0 && SF_STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 64 == 0 && HALF % 32 == 0, "tile shape");
 };
@@ -71,12 +86,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* epi_smem = smem + C::STAGE_BYTES * STAGES;
+  uint8_t* sf_smem = smem + C::STAGE_BYTES * STAGES;
+  uint8_t* epi_smem = sf_smem + C::SF_STAGE_BYTES * C::SF_STAGES;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + C::NUM_ACC;
-  uint64_t* drain = acc_empty + C::NUM_ACC;
+  uint64_t* sf_full = acc_empty + C::NUM_ACC;     // [SF_STAGES] this CTA's scale atoms landed
+  uint64_t* sf_empty = sf_full + C::SF_STAGES;    // [SF_STAGES] the scale warps have read them
+  uint64_t* tsf_ready = sf_empty + C::SF_STAGES;  // [NB_TSF] even CTA's: both CTAs' slot written
+  uint64_t* tsf_free = tsf_ready + C::NB_TSF;     // [NB_TSF] the MMAs that read the slot are done
+  uint64_t* drain = tsf_free + C::NB_TSF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -94,6 +114,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int a = 0; a < C::NUM_ACC; ++a) {
       mbar_init(smem_u32(&acc_full[a]), 1);
       mbar_init(smem_u32(&acc_empty[a]), 2 * C::EPI_WARPS);
+    }
+    for (int s = 0; s < C::SF_STAGES; ++s) {
+      mbar_init(smem_u32(&sf_full[s]), 1);
+      mbar_init(smem_u32(&sf_empty[s]), 4);
+    }
+    for (int b = 0; b < C::NB_TSF; ++b) {
+      mbar_init(smem_u32(&tsf_ready[b]), 8);
+      mbar_init(smem_u32(&tsf_free[b]), 1);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -123,12 +151,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nkb = p.K / C::BK;
   const int pair = blockIdx.x >> 1;
   const int pairs = gridDim.x >> 1;
+  // K steps (with scales) this pair runs: every tile pair, pair+pairs, ...
+  const uint32_t total_ks = pair < total ? static_cast<uint32_t>((total - 1 - pair) / pairs + 1) * nkb : 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
+      // scale atoms of K step k (counted over this pair's tiles) into slot k % SF_STAGES
+      auto issue_sf = [&](uint32_t k) -> bool {
+        const int tile = pair + static_cast<int>(k / nkb) * pairs;
+        const int kb = static_cast<int>(k % nkb);
+        const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+        const int n0 = (tile / m_tiles) * BN;
+        const uint32_t slot = k % C::SF_STAGES;
+        if (k >= static_cast<uint32_t>(C::SF_STAGES) &&
+            !mbar_wait(smem_u32(&sf_empty[slot]), ((k / C::SF_STAGES) - 1) & 1, abort_flag, p.status))
+          return false;
+        uint8_t* dst = sf_smem + slot * C::SF_STAGE_BYTES;
+        const uint32_t bar = smem_u32(&sf_full[slot]);
+        mbar_arrive_expect_tx(bar, C::SF_STAGE_BYTES);
+        tma_load_3d(smem_u32(dst), &tm_sfa, bar, 0, kb * 4, m0 / 128);
+        tma_load_3d(smem_u32(dst + C::SFA_BYTES), &tm_sfb, bar, 0, kb * 4, n0 / 128);
+        return true;
+      };
+      uint32_t ksf = 0;
+      while (ksf < total_ks && ksf < static_cast<uint32_t>(C::SF_STAGES)) ok = ok && issue_sf(ksf++);
       for (int tile = pair; tile < total && ok; tile += pairs) {
         const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
         const int n0 = (tile / m_tiles) * BN;
@@ -153,12 +202,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * C::STAGE_BYTES);
           tma_load_2d_pair(smem_u32(st), &tm_a, bar, kb * 128, m0);
           tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tm_b, bar, kb * 128, nb0);
-          tma_load_3d_pair(smem_u32(st + C::A_BYTES + C::B_BYTES), &tm_sfa, bar, 0, kb * 4, m0 / 128);
-          tma_load_3d_pair(smem_u32(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES), &tm_sfb, bar, 0, kb * 4,
-                           n0 / 128);
           ++it;
+          if (ksf < total_ks && !issue_sf(ksf++)) { ok = false; break; }
         }
       }
+      // no scale copy may still be landing when shared memory goes away
+      const uint32_t sf_first = ksf > static_cast<uint32_t>(C::SF_STAGES) ? ksf - C::SF_STAGES : 0u;
+      for (uint32_t k = sf_first; k < ksf; ++k)
+        mbar_wait_drain(smem_u32(&sf_full[k % C::SF_STAGES]), (k / C::SF_STAGES) & 1);
       // The even CTA's ring barriers count both CTAs' bytes: there, wait
       // (bounded) for the newest fills to land before shared memory goes away.
       if (leader) {
@@ -171,7 +222,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (leader && lane == 0) {
       constexpr uint32_t kIdescF4 = idesc_nvf4(256, BN);
       constexpr uint32_t kIdescBf = idesc_bf16(256, BN);
-      uint32_t it = 0, tcount = 0;
+      uint32_t it = 0, tcount = 0, ks = 0;
       for (int tile = pair; tile < total; tile += pairs) {
         const uint32_t acc = tcount % C::NUM_ACC;
         const uint32_t aph = (tcount / C::NUM_ACC) & 1;
@@ -204,29 +255,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t b = ks % C::NB_TSF;
+          if (!mbar_wait(smem_u32(&tsf_ready[b]), (ks / C::NB_TSF) & 1, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * C::STAGE_BYTES);
           const uint32_t b_base = a_base + C::A_BYTES;
-          const uint32_t sfa_base = b_base + C::B_BYTES;
-          const uint32_t sfb_base = sfa_base + C::SFA_BYTES;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tc_cp_32x128b_x4_pair(tmem + C::SFA_COL + 4 * j, smem_desc(sfa_base + 512 * j, 0, 128, kSwizzleNone));
-#pragma unroll
-            for (int rb = 0; rb < C::SFB_RB; ++rb)
-              tc_cp_32x128b_x4_pair(tmem + C::SFB_COL + 4 * C::SFB_RB * j + 4 * rb,
-                                    smem_desc(sfb_base + 2048 * rb + 512 * j, 0, 128, kSwizzleNone));
-          }
+          const uint32_t sf = tmem + C::SF_COL0 + b * C::SF_COLS;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint64_t ad = smem_desc(a_base + 32 * j, 16, 1024, kSwizzle128B);
             const uint64_t bd = smem_desc(b_base + 32 * j, 16, 1024, kSwizzle128B);
-            mma_nvf4_pair(d, ad, bd, kIdescF4, tmem + C::SFA_COL + 4 * j,
-                          tmem + C::SFB_COL + 4 * C::SFB_RB * j + sfb_shift,
+            mma_nvf4_pair(d, ad, bd, kIdescF4, sf + 4 * j, sf + 16 + 4 * C::SFB_RB * j + sfb_shift,
                           (!first || j > 0) ? 1u : 0u);
           }
           tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);
+          tc_commit_pair_mc(smem_u32(&tsf_free[b]), 0x3);
           ++it;
+          ++ks;
           first = false;
         }
         if (!ok) break;
@@ -236,7 +281,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_commit_pair(smem_u32(drain));
       mbar_wait_drain(smem_u32(drain), 0);
     }
-  } else {
+  } else if (warp < C::SF_WARP0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int ew = warp - 2;
     const int q = warp & 3;               // TMEM lane quarter (rows 32q..32q+31 of this CTA)
@@ -313,6 +358,48 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
+  } else {
+    // ------------------------------------------------------------ scale warps (both CTAs)
+    // Lane l holds, per 512-byte atom, the 16 bytes of rows l, l+32, l+64,
+    // l+96 (one 32-bit TMEM column per row); every lane quarter gets the same
+    // words, so each row's scales sit in its own lane at column 4j + row/32.
+    const int q = warp & 3;  // the TMEM lane quarter this warp may write
+    const uint32_t tsf_ready_leader0 = mapa_shared(smem_u32(&tsf_ready[0]), 0);
+    for (uint32_t k = 0; k < total_ks; ++k) {
+      const uint32_t slot = k % C::SF_STAGES;
+      const uint32_t b = k % C::NB_TSF;
+      if (!mbar_wait(smem_u32(&sf_full[slot]), (k / C::SF_STAGES) & 1, abort_flag, p.status)) break;
+      if (k >= static_cast<uint32_t>(C::NB_TSF) &&
+          !mbar_wait(smem_u32(&tsf_free[b]), ((k / C::NB_TSF) - 1) & 1, abort_flag, p.status))
+        break;
+      const uint8_t* src = sf_smem + slot * C::SF_STAGE_BYTES;
+      uint32_t v[C::SF_COLS];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src + 512 * j + 16 * lane);
+        v[4 * j] = w.x; v[4 * j + 1] = w.y; v[4 * j + 2] = w.z; v[4 * j + 3] = w.w;
+#pragma unroll
+        for (int rb = 0; rb < C::SFB_RB; ++rb) {
+          const uint4 u = *reinterpret_cast<const uint4*>(src + C::SFA_BYTES + 2048 * rb + 512 * j + 16 * lane);
+          const int c = 16 + 4 * C::SFB_RB * j + 4 * rb;
+          v[c] = u.x; v[c + 1] = u.y; v[c + 2] = u.z; v[c + 3] = u.w;
+        }
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + C::SF_COL0 + b * C::SF_COLS;
+#pragma unroll
+      for (int c = 0; c < C::SF_COLS; c += 16)
+        tmem_st_16cols(taddr + c, *reinterpret_cast<const uint32_t(*)[16]>(&v[c]));
+      tmem_st_wait();
+      // the words are in TMEM: the ring slot may be refilled (async proxy)
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&sf_empty[slot]));
+        mbar_arrive_cluster(tsf_ready_leader0 + 8 * b);
+      }
+    }
   }
 
   tc_fence_before();
