@@ -35,7 +35,7 @@
 
 namespace w4a4 {
 
-template <int BN_, int STAGES_>
+template <int BN_, int STAGES_, int SF_STAGES_ = 5, int EPI_NBUF_ = 2, bool ALIGN_BASE_ = true>
 struct Gemm2Cfg {
   static constexpr int BN = BN_;                       // tile width (output columns)
   static constexpr int BH = BN / 2;                    // B rows held by each CTA
@@ -53,7 +53,7 @@ struct Gemm2Cfg {
   static constexpr int SFB_RB = BN / 128 + (BN % 128 ? 1 : 0);
   static constexpr int SFB_BYTES = SFB_RB * 4 * 512;
   static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
-  static constexpr int SF_STAGES = 5;
+  static constexpr int SF_STAGES = SF_STAGES_;
   // TMEM: accumulator(s), then scale slots of SF_COLS columns (per K-block j
   // of the step: A scales at 4j, weight-scale block rb at 16 + 4*SFB_RB*j + 4*rb)
   static constexpr int SF_COLS = 16 + 4 * 4 * SFB_RB;
@@ -67,8 +67,17 @@ struct Gemm2Cfg {
   static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * 4;
   static constexpr int HALF = BN / 2;                  // columns per epilogue warp
   static constexpr int EPI_BUF = 32 * 64;              // 32 rows x 32 bf16, one staging buffer
-  static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
-  static constexpr int SMEM = STAGE_BYTES * STAGES + SF_STAGE_BYTES * SF_STAGES + EPI_BYTES + 1024 + 512;
+  static constexpr int EPI_NBUF = EPI_NBUF_;           // staging buffers per epilogue warp
+  static constexpr int EPI_BYTES = EPI_WARPS * EPI_NBUF * EPI_BUF;
+  // ALIGN_BASE: round the dynamic shared memory base up to 1024 bytes (costs
+  // up to 1 KB); otherwise the base must already be 1024-aligned (checked)
+  static constexpr bool ALIGN_BASE = ALIGN_BASE_;
+  // mbarriers (full/empty, accumulator, scale ring, TMEM scale slots, drain),
+  // then the TMEM address and the abort flag
+  static constexpr int BAR_BYTES = (8 * (2 * STAGES + 2 * 2 + 2 * SF_STAGES + 2 * 6 + 1) + 8 + 127) / 128 * 128;
+  static constexpr int SMEM =
+      STAGE_BYTES * STAGES + SF_STAGE_BYTES * SF_STAGES + EPI_BYTES + (ALIGN_BASE ? 1024 : 0) + BAR_BYTES;
+
   static_assert(NB_TSF >= 2 && SF_COL0 + NB_TSF * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SF_COLS % 16 == 0, "scale slot written 16 columns at a time");
   static_assert(STAGE_BYTES % 1024 == 0 && SF_STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -84,8 +93,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                  const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   constexpr int BN = C::BN, STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = C::ALIGN_BASE
+                      ? reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023))
+                      : smem_raw;
+  if (!C::ALIGN_BASE && (smem_u32(smem_raw) & 1023u) != 0) {
+    // the swizzled TMA tiles need 1024-byte alignment; every CTA sees the
+    // same base, so all return here before any barrier or TMEM use
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, kStatusMisaligned);
+    return;
+  }
   uint8_t* sf_smem = smem + C::STAGE_BYTES * STAGES;
   uint8_t* epi_smem = sf_smem + C::SF_STAGE_BYTES * C::SF_STAGES;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
@@ -288,7 +304,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int h = ew >> 2;                // column half
     const float alpha = __fmul_rn(__ldg(p.t_x), __ldg(p.t_w));
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-    uint8_t* stage_buf = epi_smem + ew * 2 * C::EPI_BUF;
+    uint8_t* stage_buf = epi_smem + ew * C::EPI_NBUF * C::EPI_BUF;
     uint32_t tcount = 0, chunk = 0;
     for (int tile = pair; tile < total; tile += pairs) {
       const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
@@ -311,10 +327,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
       for (int c = 0; c < C::HALF / 32; ++c, ++chunk) {
         const int n = n0 + h * C::HALF + 32 * c;
-        uint8_t* buf = stage_buf + (chunk & 1) * C::EPI_BUF;
-        if (chunk >= 2) {
+        uint8_t* buf = stage_buf + (chunk % C::EPI_NBUF) * C::EPI_BUF;
+        if (chunk >= static_cast<uint32_t>(C::EPI_NBUF)) {
           // the TMA store that last used this buffer has finished reading it
-          if (lane == 0) bulk_wait_group_read<1>();
+          if (lane == 0) bulk_wait_group_read<C::EPI_NBUF - 1>();
           __syncwarp();
         }
         uint32_t packed[16];

@@ -31,11 +31,15 @@ constexpr int kAmaxThreads = 256;
 constexpr int kAmaxMaxBlocks = 1024;
 constexpr int kQRows = 128;       // rows per CTA (one TMEM lane per row)
 constexpr int kQChunk = 64;       // K elements per pipeline step (one SF atom column)
-constexpr int kQComputeWarps = 4;  // one thread per row of the 128-row tile
-constexpr int kQProducerWarp = 4;  // TMA producer
-constexpr int kQMmaWarp = 5;       // TMEM owner, issues the U = X L1 MMAs
-constexpr int kQThreads = 32 * 6;
-constexpr int kQTargetCtas = 296; // two CTAs per SM on a 148-SM part
+// Two-pass quantiser (pass 2): three groups of four compute warps (one thread
+// per row of the 128-row tile, group g takes chunks g, g+3, ...), a TMA
+// producer warp and the TMEM owner / U-MMA warp; one CTA per SM.
+constexpr int kQGroups = 3;
+constexpr int kQComputeWarps = 4 * kQGroups;
+constexpr int kQProducerWarp = kQComputeWarps;      // TMA producer
+constexpr int kQMmaWarp = kQComputeWarps + 1;       // TMEM owner, issues the U = X L1 MMAs
+constexpr int kQThreads = 32 * (kQComputeWarps + 2);
+constexpr int kQTargetCtas = 592;  // about four work items per SM on a 148-SM part
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -44,11 +48,21 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ------------------------------------------------------------------ pass 1
-// A warp reads 32 consecutive 16-byte vectors of one row per work item (a
-// row segment), so the channel index of each lane needs no division; every
-// lane keeps kAmaxUnroll loads in flight.  Plain cached loads leave the
-// tensor in L2 for pass 2.
+// The tensor amax of the smoothed activation, max |fl(x_mk * s_k)|.  Rounding
+// is monotonic and s_k > 0, so it equals max over k of fl(max_m |x_mk| * s_k):
+// each thread owns one 16-byte column segment (8 bf16 or 4 fp32 channels) of a
+// band of rows, keeps the running column maxima of |x| (packed bf16x2 maxima
+// for bf16) and multiplies by s once per column at the end.  A warp reads 512
+// contiguous bytes of a row per load; every lane keeps kAmaxUnroll loads in
+// flight.  Plain cached loads leave the tensor in L2 for pass 2.
 constexpr int kAmaxUnroll = 8;
+
+// max(|a|, |b|) per bf16 half (the sign bits of the result are not used)
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 
 template <typename SrcT>
 __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restrict__ X, int64_t M,
@@ -56,69 +70,70 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restri
                                                             const float* __restrict__ inv_s,
                                                             float* __restrict__ partials,
                                                             int* __restrict__ tickets,
-                                                            int n_tickets) {
-  constexpr int EPV = 16 / sizeof(SrcT);  // elements per 16-byte vector
+                                                            int n_tickets, int rows_per_cta) {
+  constexpr int EPV = 16 / sizeof(SrcT);  // channels per 16-byte segment
   const int lane = threadIdx.x & 31;
-  const int segs = static_cast<int>(K / (32 * EPV));  // row segments (K % 256 == 0)
-  const int64_t items = M * segs;
-  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t segs = K / EPV;
+  const int64_t seg = static_cast<int64_t>(blockIdx.x) * kAmaxThreads + threadIdx.x;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
+  const int64_t r1 = r0 + rows_per_cta < M ? r0 + rows_per_cta : M;
   float m = 0.0f;
-  for (int64_t base = warp_global * kAmaxUnroll; base < items; base += warps * kAmaxUnroll) {
-    uint4 raw[kAmaxUnroll];
-    int col[kAmaxUnroll];
+  if (seg < segs) {
+    const SrcT* col = X + seg * EPV;
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};  // |x| maxima: 4 bf16x2 words or 4 fp32 bit patterns
+    for (int64_t row = r0; row < r1; row += kAmaxUnroll) {
+      uint4 raw[kAmaxUnroll];
 #pragma unroll
-    for (int u = 0; u < kAmaxUnroll; ++u) {
-      const int64_t it = base + u;
-      col[u] = -1;
-      if (it < items) {
-        const int64_t row = it / segs;
-        const int seg = static_cast<int>(it - row * segs);
-        col[u] = (seg * 32 + lane) * EPV;
-        raw[u] = __ldg(reinterpret_cast<const uint4*>(X + row * ld + col[u]));
-      }
-    }
+      for (int u = 0; u < kAmaxUnroll; ++u)
+        if (row + u < r1) raw[u] = __ldg(reinterpret_cast<const uint4*>(col + (row + u) * ld));
 #pragma unroll
-    for (int u = 0; u < kAmaxUnroll; ++u) {
-      if (col[u] < 0) continue;
-      float v[EPV];
-      if constexpr (sizeof(SrcT) == 2) {
+      for (int u = 0; u < kAmaxUnroll; ++u) {
+        if (row + u >= r1) continue;
         const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          v[2 * j] = bf16_lo(w[j]);
-          v[2 * j + 1] = bf16_hi(w[j]);
-        }
-      } else {
-        v[0] = __uint_as_float(raw[u].x);
-        v[1] = __uint_as_float(raw[u].y);
-        v[2] = __uint_as_float(raw[u].z);
-        v[3] = __uint_as_float(raw[u].w);
-      }
-      if (inv_s != nullptr) {
-#pragma unroll
-        for (int j = 0; j < EPV; j += 4) {
-          const float4 s = __ldg(reinterpret_cast<const float4*>(inv_s + col[u] + j));
-          v[j] = __fmul_rn(v[j], s.x);
-          v[j + 1] = __fmul_rn(v[j + 1], s.y);
-          v[j + 2] = __fmul_rn(v[j + 2], s.z);
-          v[j + 3] = __fmul_rn(v[j + 3], s.w);
+          if constexpr (sizeof(SrcT) == 2)
+            acc[j] = bf16x2_absmax(acc[j], w[j]);
+          else
+            acc[j] = __float_as_uint(fmaxf(__uint_as_float(acc[j]), fabsf(__uint_as_float(w[j]))));
         }
       }
-#pragma unroll
-      for (int j = 0; j < EPV; ++j) m = fmaxf(m, fabsf(v[j]));
     }
+    float v[EPV];
+    if constexpr (sizeof(SrcT) == 2) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = bf16_lo(acc[j] & 0x7FFF7FFFu);
+        v[2 * j + 1] = bf16_hi(acc[j] & 0x7FFF7FFFu);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = __uint_as_float(acc[j]);
+    }
+    if (inv_s != nullptr) {
+#pragma unroll
+      for (int j = 0; j < EPV; j += 4) {
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(inv_s + seg * EPV + j));
+        v[j] = __fmul_rn(v[j], s4.x);
+        v[j + 1] = __fmul_rn(v[j + 1], s4.y);
+        v[j + 2] = __fmul_rn(v[j + 2], s4.z);
+        v[j + 3] = __fmul_rn(v[j + 3], s4.w);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < EPV; ++j) m = fmaxf(m, v[j]);
   }
   __shared__ float red[kAmaxThreads / 32];
   m = warp_max(m);
   if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
+  const int cta = blockIdx.y * gridDim.x + blockIdx.x;
   if (threadIdx.x < 32) {
-    float v = threadIdx.x < kAmaxThreads / 32 ? red[threadIdx.x] : 0.0f;
-    v = warp_max(v);
-    if (threadIdx.x == 0) partials[blockIdx.x] = v;
+    float r = threadIdx.x < kAmaxThreads / 32 ? red[threadIdx.x] : 0.0f;
+    r = warp_max(r);
+    if (threadIdx.x == 0) partials[cta] = r;
   }
-  if (blockIdx.x == 0) {
+  if (cta == 0) {
     for (int t = threadIdx.x; t < n_tickets; t += blockDim.x) tickets[t] = 0;
   }
 }
@@ -148,13 +163,18 @@ struct QuantTile {
   // bf16: one 128 x 64 box (16 KB); fp32: two 128 x 32 boxes (32 KB).
   static constexpr int kBytes = kQRows * kQChunk * static_cast<int>(sizeof(SrcT));
   static constexpr int kBoxes = sizeof(SrcT) / 2;
-  static constexpr int kStages = sizeof(SrcT) == 2 ? 4 : 3;
+  static constexpr int kStages = sizeof(SrcT) == 2 ? 10 : 6;
   static constexpr int kL1Bytes = 32 * kQChunk * 2;  // L1t tile, 32 x 64 bf16 (4 KB)
   static constexpr int kL1Off = kBytes;
   static constexpr int kInvSOff = kBytes + (sizeof(SrcT) == 2 ? kL1Bytes : 0);  // 64 fp32 of inv_s
   static constexpr int kStageBytes = (kInvSOff + kQChunk * 4 + 1023) / 1024 * 1024;
-  static constexpr int kSmem = kStageBytes * kStages + 1024 + 256;
-  static_assert(kStageBytes * kStages + 8 * (3 * kStages + 1) + 64 <= kStageBytes * kStages + 256, "barrier area");
+  // ring, 1 KB alignment slack, barriers + scalars (512 B), the 256-entry
+  // table of code multipliers
+  static constexpr int kBarOff = kStageBytes * kStages;
+  static constexpr int kRqOff = kBarOff + 512;
+  static constexpr int kSmem = kRqOff + 1024 + 1024;
+  static_assert(8 * (3 * kStages + 1) + 4 * (2 + kQThreads / 32 + 1) <= 512, "barrier area");
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 // Read 8 consecutive source elements [8c, 8c+8) of row ``r`` from a 128-byte
@@ -177,6 +197,33 @@ __device__ __forceinline__ void load8(const uint8_t* tile, int r, int c, float (
       const float4 w = *reinterpret_cast<const float4*>(box + r * 128 + (((g & 7) ^ (r & 7)) << 4));
       v[4 * h] = w.x; v[4 * h + 1] = w.y; v[4 * h + 2] = w.z; v[4 * h + 3] = w.w;
     }
+  }
+}
+
+// Blackwell packed fp32 multiply: two IEEE round-to-nearest products.
+__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Eight smoothed values of row ``r``, elements 8u..8u+7 of a resident chunk
+// (``inv`` holds the chunk's 64 reciprocal smoothing factors).
+template <typename SrcT>
+__device__ __forceinline__ void load_unit(const uint8_t* tile, const float* inv, bool has_inv, int r, int u,
+                                          float (&v)[8]) {
+  load8<SrcT>(tile, r, u, v);
+  if (has_inv) {
+    const float4 s0 = reinterpret_cast<const float4*>(inv)[2 * u];
+    const float4 s1 = reinterpret_cast<const float4*>(inv)[2 * u + 1];
+    mul2_rn(v[0], v[1], v[0], v[1], s0.x, s0.y);
+    mul2_rn(v[2], v[3], v[2], v[3], s0.z, s0.w);
+    mul2_rn(v[4], v[5], v[4], v[5], s1.x, s1.y);
+    mul2_rn(v[6], v[7], v[6], v[7], s1.z, s1.w);
   }
 }
 
@@ -239,21 +286,22 @@ __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, 
 }
 
 template <typename SrcT>
-__global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_constant__ CUtensorMap tm_x,
+__global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                           const __grid_constant__ CUtensorMap tm_l1,
                                                           const QuantParams p) {
   using Tile = QuantTile<SrcT>;
   constexpr int S = Tile::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tile::kStageBytes * S);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tile::kBarOff);
   uint64_t* empty = full + S;
   uint64_t* mma_done = empty + S;
   uint64_t* drain = mma_done + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 6 floats
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 8);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);  // one float per warp
+  int* last_flag = reinterpret_cast<int*>(tmem_slot + 2 + kQThreads / 32);
+  float* rq_tab = reinterpret_cast<float*>(smem + Tile::kRqOff);  // 1/(dec(e) t) per scale code
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -269,7 +317,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), kQComputeWarps);
+      mbar_init(smem_u32(&empty[s]), 4);  // the four warps of the group that took the chunk
       mbar_init(smem_u32(&mma_done[s]), 1);
     }
     mbar_init(smem_u32(drain), 1);
@@ -351,90 +399,71 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
     }
   } else {
     // ------------------------------------------------------- quantise rows
-    const int row_in_tile = tid;  // compute warps are warps 0..3
+    // The code multiplier of every scale code, once per CTA (the same
+    // __frcp_rn(dec(e) * t) as a per-block computation).
+    const bool has_inv = p.inv_s != nullptr;
+    for (int e = tid; e < 256; e += 32 * kQComputeWarps)
+      rq_tab[e] = __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(e)).y, t));
+    named_bar_sync(1, 32 * kQComputeWarps);
+    const int grp = warp >> 2;
+    const int row_in_tile = tid & (kQRows - 1);
     const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
     const bool row_ok = row < p.M;
     const int64_t kbytes = p.K / 2;
-    for (int i = 0; i < n; ++i) {
+    for (int i = grp; i < n; i += kQGroups) {
       const int s = i % S;
       if (!mbar_wait(smem_u32(&full[s]), (i / S) & 1, abort_flag, p.status)) break;
       const uint8_t* tile = smem + s * Tile::kStageBytes;
+      const float* inv = reinterpret_cast<const float*>(tile + Tile::kInvSOff);
       const int kc = kc0 + i;
-
-      float x[64];
+      uint32_t cw[8];
+      uint32_t e4 = 0u;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float v[8];
-        load8<SrcT>(tile, row_in_tile, c, v);
+      for (int h = 0; h < 2; ++h) {
+        // blocks 2h and 2h+1 (elements 32h .. 32h+31 of the chunk)
+        float x[32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) x[8 * c + j] = v[j];
-      }
-      if (p.inv_s != nullptr) {
-        const float4* inv = reinterpret_cast<const float4*>(tile + Tile::kInvSOff);
+        for (int u = 0; u < 4; ++u)
+          load_unit<SrcT>(tile, inv, has_inv, row_in_tile, 4 * h + u, *reinterpret_cast<float(*)[8]>(&x[8 * u]));
+        float bm0 = 0.0f, bm1 = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 64; j += 4) {
-          const float4 sv = inv[j / 4];
-          x[j] = __fmul_rn(x[j], sv.x);
-          x[j + 1] = __fmul_rn(x[j + 1], sv.y);
-          x[j + 2] = __fmul_rn(x[j + 2], sv.z);
-          x[j + 3] = __fmul_rn(x[j + 3], sv.w);
+        for (int j = 0; j < 16; ++j) {
+          bm0 = fmaxf(bm0, fabsf(x[j]));
+          bm1 = fmaxf(bm1, fabsf(x[16 + j]));
         }
-      }
-      // four 16-element blocks: maxima first (this consumes every value read
-      // from the stage), then release the stage: the shared-memory reads are
-      // ordered before the refill's TMA writes by the proxy fence and the
-      // barrier's release/acquire.
-      float bmx[4];
+        // both blocks' scale bytes in one conversion; byte 0 = block 2h
+        const uint32_t e2 = cvt_e4m3x2(__fdiv_rn(__fmul_rn(bm1, rt), 6.0f), __fdiv_rn(__fmul_rn(bm0, rt), 6.0f)) & 0xFFFFu;
+        e4 |= e2 << (16 * h);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        float bm = 0.0f;
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t e = (e2 >> (8 * q)) & 0xFFu;
+          cw[4 * h + 2 * q] = cw[4 * h + 2 * q + 1] = 0u;
+          if (e != 0u) {  // a zero scale leaves the block's codes +0
+            const float rq = rq_tab[e];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) bm = fmaxf(bm, fabsf(x[16 * b + j]));
-        bmx[b] = bm;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-      uint32_t sf_word = 0;
-      uint32_t codes[8];
-#pragma unroll
-      for (int b = 0; b < 4; b += 2) {
-        const float bm0 = bmx[b], bm1 = bmx[b + 1];
-        const float s0 = __fdiv_rn(__fmul_rn(bm0, rt), 6.0f);
-        const float s1 = __fdiv_rn(__fmul_rn(bm1, rt), 6.0f);
-        const uint32_t e2 = cvt_e4m3x2(s1, s0);  // byte 0 = block b, byte 1 = block b+1
-        sf_word |= e2 << (8 * b);
-        const float2 sd = e4m3x2_to_f32(e2);     // .x = block b+1, .y = block b
-        const float sdb[2] = {sd.y, sd.x};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int blk = b + h;
-          if (sdb[h] > 0.0f) {
-            const float rq = __frcp_rn(__fmul_rn(sdb[h], t));
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
+            for (int uu = 0; uu < 2; ++uu) {
               float v[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(x[16 * blk + 8 * q + j], rq);
-              codes[2 * blk + q] = cvt_e2m1x8(v);
+              for (int j = 0; j < 8; j += 2)
+                mul2_rn(v[j], v[j + 1], x[16 * q + 8 * uu + j], x[16 * q + 8 * uu + j + 1], rq, rq);
+              cw[4 * h + 2 * q + uu] = cvt_e2m1x8(v);
             }
-          } else {
-            codes[2 * blk] = 0u;
-            codes[2 * blk + 1] = 0u;
           }
         }
       }
+      // Every value read from the stage has been consumed: release it (the
+      // shared-memory reads are ordered before the refill's TMA writes by the
+      // proxy fence and the barrier's release/acquire).
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
       if (row_ok) {
         uint4* dst = reinterpret_cast<uint4*>(p.q + row * kbytes + static_cast<int64_t>(kc) * 32);
-        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
       }
-      {
-        const int64_t atom = static_cast<int64_t>(rb) * chunks + kc;
-        uint32_t* sfw = reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (row_in_tile & 31) * 16 +
-                                                    (row_in_tile >> 5) * 4);
-        *sfw = sf_word;
-      }
+      const int64_t atom = static_cast<int64_t>(rb) * chunks + kc;
+      *reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (row_in_tile & 31) * 16 + (row_in_tile >> 5) * 4) = e4;
     }
   }
 
@@ -450,11 +479,12 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
     return;
   }
 
-  // U partial of this K slice (TMEM lane = row): compute warps read it out.
+  // U partial of this K slice (TMEM lane = row): warps 0-3 (one per TMEM lane
+  // quarter) read it out.
   const int row_in_tile = tid;
   const int64_t rows_pad = static_cast<int64_t>(gridDim.x) * kQRows;
   const int64_t prow = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-  if (warp < kQComputeWarps) {
+  if (warp < 4) {
     tc_fence_after();
     uint32_t u[32];
     tmem_ld_32cols(tmem + (static_cast<uint32_t>(warp * 32) << 16), u);
@@ -481,7 +511,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const __grid_consta
     *last_flag = (ticket == p.splits - 1) ? 1 : 0;
   }
   __syncthreads();
-  if (*last_flag && warp < kQComputeWarps) {
+  if (*last_flag && warp < 4) {
     const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
     finalize_lowrank(p, t, rows_pad, prow, row);
   }
@@ -525,21 +555,7 @@ constexpr int kFThreads = 32 * 16;
 static_assert(kFusedMaxChunks % kFGroups == 0, "chunk groups");
 static_assert(kFComputeWarps * 32 >= 256, "one thread per scale code fills the multiplier table");
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 static_assert(kFUWarp0 % 4 == 0 && kFThreads == 32 * (kFUWarp0 + 4), "lane quarters");
-
-// Blackwell packed fp32 multiply: two IEEE round-to-nearest products.
-__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 a, b, d;\n\t"
-      "mov.b64 a, {%2, %3};\n\t"
-      "mov.b64 b, {%4, %5};\n\t"
-      "mul.rn.f32x2 d, a, b;\n\t"
-      "mov.b64 {%0, %1}, d;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -549,10 +565,6 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 
 __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void named_bar_arrive(int id, int count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Bounded spin until a global counter reaches ``target``; false on timeout
@@ -569,25 +581,6 @@ __device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target,
     __nanosleep(64);
   }
   return true;
-}
-
-// Eight smoothed values of row ``r``, 16-byte unit ``u`` (elements 8u..8u+7)
-// of a resident bf16 chunk.
-__device__ __forceinline__ void load_unit(const uint8_t* tile, const float* inv, bool has_inv, int r, int u,
-                                          float (&v)[8]) {
-  const uint4 w = *reinterpret_cast<const uint4*>(tile + r * 128 + ((u ^ (r & 7)) << 4));
-  v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x);
-  v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
-  v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z);
-  v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
-  if (has_inv) {
-    const float4 s0 = reinterpret_cast<const float4*>(inv)[2 * u];
-    const float4 s1 = reinterpret_cast<const float4*>(inv)[2 * u + 1];
-    mul2_rn(v[0], v[1], v[0], v[1], s0.x, s0.y);
-    mul2_rn(v[2], v[3], v[2], v[3], s0.z, s0.w);
-    mul2_rn(v[4], v[5], v[4], v[5], s1.x, s1.y);
-    mul2_rn(v[6], v[7], v[6], v[7], s1.z, s1.w);
-  }
 }
 
 __global__ void __launch_bounds__(kFThreads, 1)
@@ -797,7 +790,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           float v[8];
-          load_unit(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, u, v);
+          load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, u, v);
           float bm = bmax[4 * i + u / 2];
 #pragma unroll
           for (int j = 0; j < 8; ++j) bm = fmaxf(bm, fabsf(v[j]));
@@ -859,7 +852,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
               for (int uu = 0; uu < 2; ++uu) {
                 float v[8];
-                load_unit(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
+                load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
                 mul2_rn(v[0], v[1], v[0], v[1], rq, rq);
                 mul2_rn(v[2], v[3], v[2], v[3], rq, rq);
                 mul2_rn(v[4], v[5], v[4], v[5], rq, rq);

@@ -14,6 +14,7 @@ namespace w4a4 {
 // --------------------------------------------------------------- status word
 // Device-side error codes written to the caller-visible status word.
 constexpr int kStatusTimeout = -7;
+constexpr int kStatusMisaligned = -10;
 
 // A wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz).
 constexpr long long kWaitBoundCycles = 4000000000LL;
@@ -88,6 +89,14 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - start > kWaitBoundCycles / 8) return;
   }
+}
+
+// --------------------------------------------------------------- named barriers
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // --------------------------------------------------------------- TMA

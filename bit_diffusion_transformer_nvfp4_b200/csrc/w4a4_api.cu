@@ -229,13 +229,19 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   int* tickets = reinterpret_cast<int*>(w + plan.off_tickets);
   float* upart = reinterpret_cast<float*>(w + plan.off_upart);
 
+  // pass 1: column-segment CTAs (x) times row bands (y), about four CTAs per
+  // SM, at most kAmaxMaxBlocks partial maxima
   constexpr int EPV = 16 / sizeof(SrcT);
-  const int64_t items = M * (K / (32 * EPV));  // warp work items (row segments)
-  int64_t grid1 = ceil_div(items, (kAmaxThreads / 32) * kAmaxUnroll);
-  if (grid1 > kAmaxMaxBlocks) grid1 = kAmaxMaxBlocks;
-  if (grid1 < 1) grid1 = 1;
-  amax_kernel<SrcT><<<static_cast<unsigned>(grid1), kAmaxThreads, 0, stream>>>(
-      X, M, K, ld, inv_s, partials, tickets, static_cast<int>(plan.row_blocks));
+  const int64_t gx = ceil_div(K / EPV, kAmaxThreads);
+  int64_t gy = ceil_div(4 * static_cast<int64_t>(dev->num_sms), gx);
+  if (gy > kAmaxMaxBlocks / gx) gy = kAmaxMaxBlocks / gx;
+  if (gy > M) gy = M;
+  if (gy < 1) gy = 1;
+  const int64_t rows_per = ceil_div(M, gy);
+  gy = ceil_div(M, rows_per);
+  const int64_t grid1 = gx * gy;
+  amax_kernel<SrcT><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kAmaxThreads, 0, stream>>>(
+      X, M, K, ld, inv_s, partials, tickets, static_cast<int>(plan.row_blocks), static_cast<int>(rows_per));
   if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
 
   CUtensorMap tm_x, tm_l1;
@@ -588,6 +594,7 @@ const char* w4a4_status_string(int status) {
     case W4A4_ERR_DEVICE_TIMEOUT: return "a device-side pipeline wait exceeded its bound";
     case W4A4_ERR_ARG: return "an enum argument is out of range";
     case W4A4_ERR_SCRATCH_LIMIT: return "the problem needs more scratch than the built-in no-alloc array holds";
+    case W4A4_ERR_DEVICE_LAYOUT: return "a kernel found its dynamic shared memory base misaligned";
     default: return "unknown status";
   }
 }

@@ -75,7 +75,8 @@ typedef enum {
   W4A4_ERR_CUDA = -6,           /* a CUDA call or kernel launch failed */
   W4A4_ERR_DEVICE_TIMEOUT = -7, /* sticky device status: a bounded wait gave up */
   W4A4_ERR_ARG = -8,            /* an enum argument is out of range */
-  W4A4_ERR_SCRATCH_LIMIT = -9   /* problem needs more than the built-in scratch (no-alloc entry) */
+  W4A4_ERR_SCRATCH_LIMIT = -9,  /* problem needs more than the built-in scratch (no-alloc entry) */
+  W4A4_ERR_DEVICE_LAYOUT = -10  /* sticky device status: a kernel found its shared memory misaligned */
 } w4a4_status;
 
 enum { W4A4_EPI_NONE = 0, W4A4_EPI_GELU_TANH = 1 };
@@ -199,7 +200,7 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
                                uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* stream);
 
 /* Copies the sticky device status word of the current device into *status
- * (W4A4_OK or W4A4_ERR_DEVICE_TIMEOUT) and clears it if reset != 0.  This call
+ * (W4A4_OK, W4A4_ERR_DEVICE_TIMEOUT or W4A4_ERR_DEVICE_LAYOUT) and clears it if reset != 0.  This call
  * synchronises the device.  Returns W4A4_OK or W4A4_ERR_CUDA. */
 int w4a4_device_status(int* status, int reset);
 

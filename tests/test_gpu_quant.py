@@ -149,3 +149,25 @@ def test_quant_lowrank_stage_reuse(w4, M, K):
     assert torch.equal(qa.Xq, qb.Xq) and torch.equal(qa.Xsf, qb.Xsf) and torch.equal(qa.U, qb.U)
     check_bytes(c.x, p["inv_s"], qa.Xq.cpu().numpy(), sf_atoms_to_rowmajor(qa.Xsf.cpu().numpy(), M, K),
                 float(qa.t_x.cpu()[0]))
+
+
+def test_quant_two_pass_full_size(w4):
+    """The 12288-deep MLP down-projection input (4608 x 12288) needs more K
+    slices than can be co-resident, so it takes the two-pass quantiser
+    (column-maxima amax pass, then the grouped quantise pass with the U MMAs
+    and the cross-slice U sums): every code and scale byte bit for bit, U on
+    sampled rows within fp32 rounding."""
+    c = config_cases(3)[1]
+    g = rng(33)
+    inv_s = (1.0 / np.exp(0.3 * g.standard_normal(c.K))).astype(np.float32)
+    L1t = bf16_round((g.standard_normal((32, c.K)) * 0.02).astype(np.float32))
+    t_w = 0.01
+    qa, xq, sf, t = run_quant(w4, c.x, inv_s, L1t, t_w)
+    check_bytes(c.x, inv_s, xq, sf, t)
+    rows = np.sort(g.choice(c.M, 256, replace=False))
+    rows[-1] = c.M - 1
+    U = qa.U.float().cpu().numpy()[rows]
+    got = U[:, :32].astype(np.float64) + U[:, 32:].astype(np.float64)
+    alpha = np.float64(np.float32(np.float32(t) * np.float32(t_w)))
+    ref = olinear.lowrank_down(c.x[rows], L1t) / alpha  # U uses the raw X and L1t as given
+    assert olinear.rel_frobenius(got, ref) < 1e-5
