@@ -37,9 +37,13 @@ _SIG = {
     "w4a4_workspace_bytes": (_c.c_size_t, [_I64, _I64, _I64, _c.c_int]),
     "nvfp4_quantize_act": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P, _P,
                                       _c.c_size_t, _P]),
+    "nvfp4_quantize_act_with_amax": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P,
+                                                _P, _P, _c.c_size_t, _P]),
     "nvfp4_pack_weight": (_c.c_int, [_P, _c.c_int, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_size_t, _P]),
     "w4a4_gemm": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _c.c_int,
                              _P, _I64, _P]),
+    "w4a4_gemm_next_amax": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P,
+                                       _c.c_int, _P, _I64, _P, _P, _P]),
     "w4a4_linear": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _c.c_int, _P, _c.c_int, _P,
                                _P, _c.c_size_t, _P]),
     "w4a4_device_status": (_c.c_int, [_c.POINTER(_c.c_int), _c.c_int]),
@@ -115,6 +119,14 @@ def nvfp4_quantize_act(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, worksp
         _stream(stream)))
 
 
+def nvfp4_quantize_act_with_amax(X, M, K, ldx, inv_s, L1t, r, t_w, amax, Xq, Xsf, t_x, U, workspace,
+                                 stream=None):
+    _check("nvfp4_quantize_act_with_amax", lib().nvfp4_quantize_act_with_amax(
+        _ptr(X), M, K, ldx, _ptr(inv_s), _ptr(L1t), r, _ptr(t_w), _ptr(amax), _ptr(Xq), _ptr(Xsf), _ptr(t_x),
+        _ptr(U), _ptr(workspace), workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream(stream)))
+
+
 def nvfp4_pack_weight(R, src_dtype, N, K, ldr, Wq, Wsf, t_w, workspace, stream=None):
     _check("nvfp4_pack_weight", lib().nvfp4_pack_weight(
         _ptr(R), src_dtype, N, K, ldr, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(workspace),
@@ -125,6 +137,13 @@ def w4a4_gemm(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y,
     _check("w4a4_gemm", lib().w4a4_gemm(
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), epilogue, _ptr(Y), ldy, _stream(stream)))
+
+
+def w4a4_gemm_next_amax(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, next_inv_s,
+                        next_amax, stream=None):
+    _check("w4a4_gemm_next_amax", lib().w4a4_gemm_next_amax(
+        _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
+        _ptr(bias), epilogue, _ptr(Y), ldy, _ptr(next_inv_s), _ptr(next_amax), _stream(stream)))
 
 
 def w4a4_linear(X, M, N, K, Wq, Wsf, t_w, inv_s, L1t, L2t, r, bias, epilogue, Y, workspace, stream=None):
@@ -179,7 +198,9 @@ class PackedWeight:
                             None if self.bias is None else self.bias[r0:r1])
 
 
-def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None) -> QuantizedActivation:
+def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None, amax=None) -> QuantizedActivation:
+    """NVFP4 activation quantisation; ``amax`` (fp32 device scalar, e.g. from
+    ``gemm(..., next_amax=...)``) supplies the tensor amax instead of measuring it."""
     M, K = X.shape
     r = 0 if L1t is None else int(L1t.shape[0])
     dev = X.device
@@ -188,7 +209,10 @@ def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None) -
     t_x = torch.empty(1, dtype=torch.float32, device=dev)
     U = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev) if r else None
     ws = _u8(max(16, nvfp4_quant_workspace_bytes(M, K, r)), dev)
-    nvfp4_quantize_act(X, M, K, X.stride(0), inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, ws, stream)
+    if amax is None:
+        nvfp4_quantize_act(X, M, K, X.stride(0), inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, ws, stream)
+    else:
+        nvfp4_quantize_act_with_amax(X, M, K, X.stride(0), inv_s, L1t, r, t_w, amax, Xq, Xsf, t_x, U, ws, stream)
     return QuantizedActivation(Xq, Xsf, t_x, U, M, K, r)
 
 
@@ -204,11 +228,19 @@ def pack_weight(R: torch.Tensor, inv_s=None, L1t=None, L2t=None, bias=None, stre
     return PackedWeight(Wq, Wsf, t_w, N, K, inv_s, L1t, L2t, bias)
 
 
-def gemm(qa: QuantizedActivation, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, stream=None):
+def gemm(qa: QuantizedActivation, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, stream=None,
+         next_inv_s=None, next_amax=None):
+    """Y = the fused W4A4 GEMM.  With ``next_amax`` (fp32 device scalar holding
+    a non-negative value, normally 0) it also max-es in the tensor amax
+    max |fl(Y * next_inv_s)| that the next layer's quantiser needs."""
     if Y is None:
         Y = torch.empty(qa.M, w.N, dtype=torch.bfloat16, device=qa.Xq.device)
-    w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias,
-              epilogue, Y, Y.stride(0), stream)
+    if next_amax is None:
+        w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias,
+                  epilogue, Y, Y.stride(0), stream)
+    else:
+        w4a4_gemm_next_amax(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias,
+                            epilogue, Y, Y.stride(0), next_inv_s, next_amax, stream)
     return Y
 
 

@@ -47,7 +47,42 @@ struct GemmParams {
   int has_lr;
   int epi;
   int* status;
+  // optional: the next layer's tensor amax max |fl(y * next_inv_s)| over the
+  // stored bf16 outputs, atomically max-ed into *next_amax (as float bits;
+  // non-negative floats order like their bit patterns).  next_inv_s may be
+  // null (all ones).
+  const float* next_inv_s;
+  unsigned* next_amax;
 };
+
+// Fold eight stored bf16 outputs (columns n .. n+7) into a running amax of
+// |y * s| (s > 0, so |fl(y s)| = fl(|y| s)).
+__device__ __forceinline__ float amax_fold8(float m, uint4 o, const float* next_inv_s, int n) {
+  const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[2 * j] = fabsf(bf16_lo(w[j]));
+    v[2 * j + 1] = fabsf(bf16_hi(w[j]));
+  }
+  if (next_inv_s != nullptr) {
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(next_inv_s + n));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(next_inv_s + n + 4));
+    v[0] = __fmul_rn(v[0], s0.x); v[1] = __fmul_rn(v[1], s0.y); v[2] = __fmul_rn(v[2], s0.z);
+    v[3] = __fmul_rn(v[3], s0.w); v[4] = __fmul_rn(v[4], s1.x); v[5] = __fmul_rn(v[5], s1.y);
+    v[6] = __fmul_rn(v[6], s1.z); v[7] = __fmul_rn(v[7], s1.w);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m = fmaxf(m, v[j]);
+  return m;
+}
+
+// One atomic max per warp of the lanes' running maxima.
+__device__ __forceinline__ void amax_publish(float m, unsigned* next_amax) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0 && next_amax != nullptr) atomicMax(next_amax, __float_as_uint(m));
+}
 
 template <int BN_, int STAGES_>
 struct GemmCfg {
@@ -74,10 +109,20 @@ struct GemmCfg {
   static_assert(HALF % 32 == 0, "epilogue column split");
 };
 
+// GELU, tanh form: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715 y^3),
+// with the hardware tanh (tanh.approx.f32, relative error about 2^-11, far
+// inside the bf16 rounding of the result).  No division: the earlier
+// y / (1 + exp(-2u)) form took the IEEE division's slow path whenever exp
+// overflowed (large negative y), which made the epilogue the bottleneck.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float r;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 __device__ __forceinline__ float gelu_tanh_f32(float y) {
-  // 0.5 y (1 + tanh(u)) == y / (1 + exp(-2u)),  u = sqrt(2/pi) (y + 0.044715 y^3)
   const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
-  return y / (1.0f + __expf(-2.0f * u));
+  const float hy = 0.5f * y;
+  return fmaf(hy, tanh_approx(u), hy);
 }
 
 template <class C>
@@ -249,6 +294,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int h = (warp - 2) >> 2;        // column half
     const float alpha = __fmul_rn(__ldg(p.t_x), __ldg(p.t_w));
+    float amax = 0.0f;  // next layer's amax over this thread's stored outputs
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const int m0 = (tile % m_tiles) * C::BM;
@@ -295,11 +341,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             o.z = pack_bf16x2(y[4], y[5]);
             o.w = pack_bf16x2(y[6], y[7]);
             *reinterpret_cast<uint4*>(yrow + n) = o;
+            if (p.next_amax != nullptr) amax = amax_fold8(amax, o, p.next_inv_s, n);
           }
         }
       }
       ++tcount;
     }
+    if (p.next_amax != nullptr) amax_publish(amax, p.next_amax);
   }
 
   tc_fence_before();

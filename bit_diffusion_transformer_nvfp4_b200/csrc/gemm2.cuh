@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const float alpha = __fmul_rn(__ldg(p.t_x), __ldg(p.t_w));
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     uint8_t* stage_buf = epi_smem + ew * C::EPI_NBUF * C::EPI_BUF;
+    float amax = 0.0f;  // next layer's amax over this thread's stored outputs
     uint32_t tcount = 0, chunk = 0;
     for (int tile = pair; tile < total; tile += pairs) {
       const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
@@ -363,6 +364,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
               make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
         }
+        if (p.next_amax != nullptr) {
+          // next layer's amax over the staged chunk (only outputs the TMA
+          // store keeps: rows < M, columns < N).  Lane l takes columns 2(l%16),
+          // 2(l%16)+1 of rows 16(l/16) .. +15: packed maxima of |y| down the
+          // column pair, then one multiply by the next 1/s per column.
+          __syncwarp();
+          const int cpair = lane & 15;
+          const int rbase = (lane >> 4) * 16;
+          uint32_t mx = 0u;
+#pragma unroll
+          for (int rr = 0; rr < 16; ++rr) {
+            const int row = rbase + rr;
+            if (row0 + row < p.M) {
+              const int phys = (cpair >> 2) ^ ((row >> 1) & 3);
+              mx = bf16x2_absmax(mx, *reinterpret_cast<const uint32_t*>(buf + row * 64 + phys * 16 + (cpair & 3) * 4));
+            }
+          }
+          const int col = n + 2 * cpair;
+          if (col < p.N) {  // N % 8 == 0: both columns of the pair are valid
+            float v0 = bf16_lo(mx & 0x7FFF7FFFu), v1 = bf16_hi(mx & 0x7FFF7FFFu);
+            if (p.next_inv_s != nullptr) {
+              const float2 s2 = __ldg(reinterpret_cast<const float2*>(p.next_inv_s + col));
+              v0 = __fmul_rn(v0, s2.x);
+              v1 = __fmul_rn(v1, s2.y);
+            }
+            amax = fmaxf(amax, fmaxf(v0, v1));
+          }
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -372,6 +401,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       ++tcount;
     }
+    if (p.next_amax != nullptr) amax_publish(amax, p.next_amax);
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   } else {

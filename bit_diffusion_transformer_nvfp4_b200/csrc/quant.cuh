@@ -57,12 +57,6 @@ __device__ __forceinline__ float warp_max(float v) {
 // flight.  Plain cached loads leave the tensor in L2 for pass 2.
 constexpr int kAmaxUnroll = 8;
 
-// max(|a|, |b|) per bf16 half (the sign bits of the result are not used)
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
 
 template <typename SrcT>
 __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restrict__ X, int64_t M,

@@ -269,7 +269,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on an mbarrier that may live in another CTA of the cluster.
 // Arrive on an mbarrier of a CTA in this cluster (default semantics: release
 // at CTA scope).  The cluster-scope release form costs the arriving thread
 // about 0.7 us per arrive here; what these arrives order is TMEM traffic,
@@ -382,6 +381,13 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
       : "=r"(r)
       : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
   return r;
+}
+
+// max(|a|, |b|) per bf16 half (the sign bits of the result are not used)
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -218,10 +218,14 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
 template <typename SrcT>
 int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* inv_s, const void* L1t, int r,
                  const float* t_w, uint8_t* q, uint8_t* sf, float* t_out, void* U, void* ws,
-                 cudaStream_t stream, DeviceInfo* dev) {
+                 cudaStream_t stream, DeviceInfo* dev, const float* amax_in = nullptr) {
+  // With the tensor amax given (by the producer of X), the quantise pass
+  // alone streams X once at any size.
   if constexpr (sizeof(SrcT) == 2) {
-    const int st = launch_quant_fused(X, M, K, ld, inv_s, L1t, r, t_w, q, sf, t_out, U, ws, stream, dev);
-    if (st != -1) return st;
+    if (amax_in == nullptr) {
+      const int st = launch_quant_fused(X, M, K, ld, inv_s, L1t, r, t_w, q, sf, t_out, U, ws, stream, dev);
+      if (st != -1) return st;
+    }
   }
   const QuantPlan plan = quant_plan(M, K, r);
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -240,9 +244,17 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   const int64_t rows_per = ceil_div(M, gy);
   gy = ceil_div(M, rows_per);
   const int64_t grid1 = gx * gy;
-  amax_kernel<SrcT><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kAmaxThreads, 0, stream>>>(
-      X, M, K, ld, inv_s, partials, tickets, static_cast<int>(plan.row_blocks), static_cast<int>(rows_per));
-  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  if (amax_in == nullptr) {
+    amax_kernel<SrcT><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kAmaxThreads, 0, stream>>>(
+        X, M, K, ld, inv_s, partials, tickets, static_cast<int>(plan.row_blocks), static_cast<int>(rows_per));
+    if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  } else if (r > 0) {
+    // the amax pass would have zeroed the U tickets
+    if (cudaMemsetAsync(tickets, 0, sizeof(int) * static_cast<size_t>(plan.row_blocks), stream) != cudaSuccess) {
+      cudaGetLastError();
+      return W4A4_ERR_CUDA;
+    }
+  }
 
   CUtensorMap tm_x, tm_l1;
   const bool is_bf16 = sizeof(SrcT) == 2;
@@ -261,8 +273,8 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   p.M = M;
   p.K = K;
   p.inv_s = inv_s;
-  p.partials = partials;
-  p.n_partials = static_cast<int>(grid1);
+  p.partials = amax_in != nullptr ? amax_in : partials;
+  p.n_partials = amax_in != nullptr ? 1 : static_cast<int>(grid1);
   p.t_w = t_w;
   p.q = q;
   p.sf = sf;
@@ -284,7 +296,8 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
 template <class C>
 int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                     int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
-                    const void* bias, int epi, void* Y, int64_t ldy, cudaStream_t stream, DeviceInfo* dev) {
+                    const void* bias, int epi, void* Y, int64_t ldy, const float* next_inv_s, unsigned* next_amax,
+                    cudaStream_t stream, DeviceInfo* dev) {
   CUtensorMap ta, tb, tsa, tsb, tu, tl;
   if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(K / 2), 128u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -317,6 +330,8 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   p.has_lr = r > 0 ? 1 : 0;
   p.epi = epi;
   p.status = dev->status_ptr;
+  p.next_inv_s = next_inv_s;
+  p.next_amax = next_amax;
   const int64_t tiles = ceil_div(M, C::BM) * ceil_div(N, C::BN);
   const int64_t grid = tiles < dev->num_sms ? tiles : dev->num_sms;
   gemm_kernel<C><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, stream>>>(ta, tb, tsa, tsb, tu, tl, p);
@@ -328,7 +343,8 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
 template <class C>
 int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                      int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
-                     const void* bias, int epi, void* Y, int64_t ldy, cudaStream_t stream, DeviceInfo* dev) {
+                     const void* bias, int epi, void* Y, int64_t ldy, const float* next_inv_s, unsigned* next_amax,
+                     cudaStream_t stream, DeviceInfo* dev) {
   CUtensorMap ta, tb, tsa, tsb, tu, tl, ty;
   if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(K / 2), 128u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -364,6 +380,8 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   p.has_lr = r > 0 ? 1 : 0;
   p.epi = epi;
   p.status = dev->status_ptr;
+  p.next_inv_s = next_inv_s;
+  p.next_amax = next_amax;
   const int64_t tiles = ceil_div(M, 2 * C::BM) * ceil_div(N, C::BN);
   const int64_t max_pairs = dev->num_sms / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -429,9 +447,9 @@ size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
   return b;
 }
 
-int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, const float* inv_s, const void* L1t, int r,
-                       const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+static int quantize_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, const float* inv_s, const void* L1t,
+                             int r, const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* workspace,
+                             size_t workspace_bytes, void* stream, const float* amax_in) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
   if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;
@@ -445,7 +463,24 @@ int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, const f
   if (st != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
   return launch_quant<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf,
-                                     t_x, U, workspace, static_cast<cudaStream_t>(stream), dev);
+                                     t_x, U, workspace, static_cast<cudaStream_t>(stream), dev, amax_in);
+}
+
+int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx, const float* inv_s, const void* L1t, int r,
+                       const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return quantize_act_impl(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, workspace, workspace_bytes, stream,
+                           nullptr);
+}
+
+int nvfp4_quantize_act_with_amax(const void* X, int64_t M, int64_t K, int64_t ldx, const float* inv_s,
+                                 const void* L1t, int r, const float* t_w, const float* amax, uint8_t* Xq,
+                                 uint8_t* Xsf, float* t_x, void* U, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!amax) return W4A4_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(amax) % 4 != 0) return W4A4_ERR_ALIGN;
+  return quantize_act_impl(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, workspace, workspace_bytes, stream,
+                           amax);
 }
 
 int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_t ldr, uint8_t* Wq, uint8_t* Wsf,
@@ -469,9 +504,10 @@ int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_
                              nullptr, workspace, s, dev);
 }
 
-int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N, int64_t K,
-              const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r, const void* bias,
-              int epilogue, void* Y, int64_t ldy, void* stream) {
+static int gemm_dispatch(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                         int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                         const void* bias, int epilogue, void* Y, int64_t ldy, const float* next_inv_s,
+                         unsigned* next_amax, void* stream) {
   int st = check_gemm_args(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy);
   if (st != W4A4_OK) return st;
   DeviceInfo* dev = nullptr;
@@ -483,12 +519,30 @@ int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const voi
   // single-CTA 128 x 192 / 128 x 256 tiles for a single row block.
   if (M > 128)
     return launch_gemm_pair<Gemm2Cfg<256, 5>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
-                                              s, dev);
+                                              next_inv_s, next_amax, s, dev);
   if (N % 192 == 0)
     return launch_gemm_cfg<GemmCfg<192, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
-                                            s, dev);
-  return launch_gemm_cfg<GemmCfg<256, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, s,
-                                          dev);
+                                            next_inv_s, next_amax, s, dev);
+  return launch_gemm_cfg<GemmCfg<256, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
+                                          next_inv_s, next_amax, s, dev);
+}
+
+int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N, int64_t K,
+              const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r, const void* bias,
+              int epilogue, void* Y, int64_t ldy, void* stream) {
+  return gemm_dispatch(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, nullptr, nullptr,
+                       stream);
+}
+
+int w4a4_gemm_next_amax(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                        int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                        const void* bias, int epilogue, void* Y, int64_t ldy, const float* next_inv_s,
+                        float* next_amax, void* stream) {
+  if (!next_amax) return W4A4_ERR_NULL;
+  if ((next_inv_s && !aligned16(next_inv_s)) || reinterpret_cast<uintptr_t>(next_amax) % 4 != 0)
+    return W4A4_ERR_ALIGN;
+  return gemm_dispatch(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, next_inv_s,
+                       reinterpret_cast<unsigned*>(next_amax), stream);
 }
 
 int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,

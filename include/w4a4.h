@@ -113,12 +113,30 @@ size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  *   U      out  bf16 [M, 2r] hi/lo low-rank activations (NULL iff r == 0)
  *   workspace   >= nvfp4_quant_workspace_bytes(M, K, r) bytes of device memory,
  *               contents need not be initialised; must not overlap the outputs
- * Launches two kernels (tensor amax, then quantise + down-projection).
+ * Launches one cooperative kernel (tensor amax, grid barrier, quantise and
+ * down-projection) when every (128-row block, K slice) tile of X fits on the
+ * device at once, otherwise two (tensor amax, then quantise + down-projection).
  */
 int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx,
                        const float* inv_s, const void* L1t, int r, const float* t_w,
                        uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_quantize_act_with_amax -- nvfp4_quantize_act with the activation's
+ * tensor amax A = max |fl(x * inv_s)| supplied by the caller (normally
+ * written by w4a4_gemm_next_amax, the producer of X) instead of measured: the
+ * quantiser then streams X once at any size.  The result is bit-identical to
+ * nvfp4_quantize_act when *amax equals the measured amax.  Same arguments as
+ * nvfp4_quantize_act plus
+ *   amax  in  fp32 device scalar (4-byte aligned), A >= 0
+ * W4A4_ERR_NULL if amax is NULL, W4A4_ERR_ALIGN if misaligned.  Launches one
+ * quantise kernel (preceded by a small memset when r > 0).
+ */
+int nvfp4_quantize_act_with_amax(const void* X, int64_t M, int64_t K, int64_t ldx,
+                                 const float* inv_s, const void* L1t, int r, const float* t_w,
+                                 const float* amax, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * nvfp4_pack_weight -- offline NVFP4 packing of the residual weight R [N, K]
@@ -152,6 +170,27 @@ int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const voi
               const uint8_t* Wq, const uint8_t* Wsf, const float* t_w,
               const void* L2t, int r, const void* bias, int epilogue,
               void* Y, int64_t ldy, void* stream);
+
+/*
+ * w4a4_gemm_next_amax -- w4a4_gemm that also measures the tensor amax the
+ * next layer's activation quantiser needs when Y is that activation (the
+ * fused producer epilogue of "NVIDIA Technical Blog Details FLUX 3 Image Klein
+ * Blackwell Inference Optimization Methods": NVFP4 with fused GEMM
+ * epilogues): over the stored bf16 outputs (after bias and GELU),
+ *   *next_amax = max(*next_amax, max_{m,n} |fl(Y[m,n] * next_inv_s[n])|)
+ * as an atomic maximum on the value's bit pattern.  Same arguments as
+ * w4a4_gemm plus
+ *   next_inv_s  in     fp32 [N] reciprocal smoothing factors of the next
+ *                      layer (> 0), 16-byte aligned, or NULL for all ones
+ *   next_amax   in/out fp32 device scalar, 4-byte aligned; must hold a
+ *                      non-negative value on entry (normally 0)
+ * W4A4_ERR_NULL if next_amax is NULL, W4A4_ERR_ALIGN if misaligned.
+ */
+int w4a4_gemm_next_amax(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U,
+                        int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,
+                        const float* t_w, const void* L2t, int r, const void* bias, int epilogue,
+                        void* Y, int64_t ldy, const float* next_inv_s, float* next_amax,
+                        void* stream);
 
 /*
  * w4a4_linear -- the whole hot path: nvfp4_quantize_act on X (row stride K)
