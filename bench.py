@@ -34,6 +34,7 @@ WORKLOAD = {"workload": "FLUX-1024px QKV projection", "M": 4608, "K": 3072, "N":
             "bias": True, "activation": "N(0,1) with 1% Student-t(2)x50 channels", "weight": "N(0,0.02)"}
 METRIC = "W4A4 linear TFLOPS (act-quant+FP4 GEMM+low-rank)"
 L2_SETS = 3          # rotating buffer sets, each ~140 MB, so every step starts L2-cold
+MID_EVERY = 10       # steps between per-kernel timing events inside the timed region
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -167,7 +168,7 @@ def build_inputs(torch, w4, prep, dev):
             torch.empty(w4.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev),
             torch.empty(1, dtype=torch.float32, device=dev),
             torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev), M, K, r)
-        ws = torch.empty(w4.nvfp4_quant_workspace_bytes(M, K, r), dtype=torch.uint8, device=dev)
+        ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         sets.append((X, w, qa, ws, Y))
     return case, x_host, sets
@@ -228,18 +229,23 @@ def run_ours(args):
     for i in range(args.warmup):
         step(i)
     barrier()
+    # Every step is bracketed by events; every MID_EVERY-th step also records
+    # one between the quantiser and the GEMM (for the per-kernel durations).
+    # An event there makes that GEMM wait for the quantiser to finish instead
+    # of starting its set-up early (programmatic launch), so the other steps
+    # go without it.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_wall0 = time.time()
     for i in range(args.steps):
         evs[i][0].record(stream)
-        step(i, evs[i][1])
+        step(i, evs[i][1] if i % MID_EVERY == 0 else None)
         evs[i][2].record(stream)
     barrier()
     t_wall1 = time.time()
     total_ms = evs[0][0].elapsed_time(evs[-1][2])
-    gemm_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    quant_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    gemm_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(0, args.steps, MID_EVERY)]
+    quant_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(0, args.steps, MID_EVERY)]
 
     # end to end through the public API with host buffers: pinned X in,
     # linear on the device, pinned Y out, every step
@@ -248,7 +254,7 @@ def run_ours(args):
     yh = _t.empty(M, N, dtype=_t.bfloat16).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
     X0, w0, qa0, ws0, Y0 = sets[0]
-    lin_ws = torch.empty(w4.w4a4_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    lin_ws = w4.new_workspace(w4.w4a4_workspace_bytes(M, N, K, r), dev)
     for i in range(2):
         X0.copy_(xh, non_blocking=True)
         w4.w4a4_linear(X0, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y0, lin_ws, stream)
@@ -295,12 +301,12 @@ def run_ours(args):
                      "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
                      "peak_kind": f"{peak_kind} (bf16 burst x4)", "launch_ms": round(gemm_avg_ms, 5),
                      "algorithmic_flops_per_launch": g_fl},
-        "kernels_ms": {"amax+quant": round(statistics.mean(quant_ms), 5), "gemm": round(gemm_avg_ms, 5)},
+        "kernels_ms": {"amax+quant": round(statistics.mean(quant_ms), 5), "gemm": round(gemm_avg_ms, 5),
+                       "sampled_steps": len(gemm_ms)},
         "e2e": {"value": round(whole_job_tflops(world, fl, 1, e2e_ms), 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2),
                 "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear"},
-        # per step: the single-pass quantiser and the pair GEMM (the
-        # quantiser's small memset is a driver copy, not a kernel of ours)
+        # per step: the single-pass quantiser and the pair GEMM
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "wall_s_timed": round(t_wall1 - t_wall0, 3),
@@ -312,6 +318,268 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- per-configuration table
+
+def run_table(args):
+    """Every configuration's layers at full size on one GPU (not the contract
+    line): per-kernel device times with L2 flushed before each repetition,
+    the whole linear (quantiser + GEMM, one event pair around both), the GEMM
+    back to back with warm L2, the MLP block (with the activation amax measured
+    by the quantiser or taken from the up-projection's epilogue), config 1 by
+    CUDA graph replay, and the denoising block per step and over a 50-step
+    trajectory at batch 1, 2 and 4.  One JSON line per row."""
+    import torch
+    import bit_diffusion_transformer_nvfp4_b200 as w4
+    from bit_diffusion_transformer_nvfp4_b200 import prep
+    from synth import bf16_bits, config_cases, trajectory_step_activation
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w4.lib()
+    s = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_kind = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    reps = args.table_reps
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(bf16_bits(a).view(np.int16))).to(dev).view(torch.bfloat16)
+
+    def med_us(fns, cold=True):
+        """Median device time (us) of each callable in ``fns`` run in sequence,
+        one event pair per callable."""
+        for _ in range(3):
+            for f in fns:
+                f()
+        torch.cuda.synchronize()
+        ts = [[] for _ in fns]
+        for _ in range(reps):
+            if cold:
+                flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            ev[0].record(s)
+            for i, f in enumerate(fns):
+                f()
+                ev[i + 1].record(s)
+            torch.cuda.synchronize()
+            for i in range(len(fns)):
+                ts[i].append(ev[i].elapsed_time(ev[i + 1]) * 1e3)
+        return [statistics.median(t) for t in ts]
+
+    def b2b_us(fn, n=20):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(n):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n * 1e3
+
+    def tf(fl, us):
+        return round(fl / (us * 1e-6) / 1e12, 1)
+
+    def check():
+        st = w4.w4a4_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {w4.w4a4_status_string(st)}")
+
+    def emit(row):
+        print(json.dumps(row), flush=True)
+
+    def prepare(case, bias=True):
+        W = dev_bf16(case.w)
+        Xc = dev_bf16(case.x_cal)
+        b = dev_bf16(case.bias) if (bias and case.bias is not None) else None
+        pk = prep.svdquant_prepare(W, Xc, r=case.r, bias=b)
+        del W, Xc
+        return pk
+
+    def linear_row(cfg, case, pk, X, epi=0):
+        M, K, N, r = X.shape[0], X.shape[1], pk.N, pk.r
+        ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
+        qa = w4.quantize_act(X, pk.inv_s, pk.L1t, pk.t_w, workspace=ws)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+        def qi():
+            w4.nvfp4_quantize_act(X, M, K, X.stride(0), pk.inv_s, pk.L1t, r, pk.t_w, qa.Xq, qa.Xsf, qa.t_x,
+                                  qa.U, ws, s)
+
+        def g():
+            w4.gemm(qa, pk, epilogue=epi, Y=Y)
+
+        def both():
+            qi()
+            g()
+        tq, tg = med_us([qi, g])
+        (tl,) = med_us([both])
+        tgb = b2b_us(g)
+        check()
+        fl = flops_per_step(M, K, N, r)
+        gfl = gemm_flops(M, K, N, r)
+        qbytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * M * 2 * r
+        row = {"table": "linear", "config": cfg, "layer": case.name, "M": M, "K": K, "N": N, "r": r,
+               "epilogue": "gelu_tanh" if epi else "none",
+               "quant_us": round(tq, 2), "quant_gbs": round(qbytes / (tq * 1e-6) / 1e9, 1),
+               "quant_frac_hbm": round(qbytes / (tq * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+               "gemm_us": round(tg, 2), "gemm_tflops": tf(gfl, tg), "gemm_frac_fp4": round(tf(gfl, tg) / fp4_peak, 3),
+               "gemm_warm_b2b_us": round(tgb, 2), "gemm_warm_b2b_tflops": tf(gfl, tgb),
+               "linear_us": round(tl, 2), "linear_tflops": tf(fl, tl),
+               "linear_frac_fp4": round(tf(fl, tl) / fp4_peak, 3)}
+        emit(row)
+        return qa, ws, Y, qi, g
+
+    emit({"table": "peaks", "fp4_peak_tflops": round(fp4_peak, 1), "hbm_gbs": peaks["hbm_gbs"],
+          "basis": f"{peak_kind}: bf16 burst x {FP4_OVER_BF16:g}; copy bandwidth", "reps": reps,
+          "l2": "256 MB buffer zeroed before each repetition"})
+
+    def graph_row(case, pk, X, qa, ws, Y, qi, g):
+        """The small layer is launch-bound: quantiser + GEMM replayed as one CUDA graph."""
+        M, K, N, r = case.M, case.K, pk.N, pk.r
+
+        def enqueue(st):
+            w4.nvfp4_quantize_act(X, M, K, K, pk.inv_s, pk.L1t, r, pk.t_w, qa.Xq, qa.Xsf, qa.t_x, qa.U, ws, st)
+            w4.w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, pk.Wq, pk.Wsf, pk.t_w, pk.L2t, r, pk.bias, 0, Y,
+                         N, st)
+
+        fl = flops_per_step(M, K, N, r)
+        (tpl,) = med_us([lambda: (qi(), g())], cold=False)
+        row = {"table": "graph", "config": 1, "layer": case.name, "linear_plain_warm_us": round(tpl, 2),
+               "linear_plain_warm_tflops": tf(fl, tpl)}
+        try:
+            side = torch.cuda.Stream()
+            side.wait_stream(s)
+            with torch.cuda.stream(side):
+                for _ in range(3):
+                    enqueue(side)
+            s.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                enqueue(torch.cuda.current_stream())
+            tgr = b2b_us(graph.replay, n=200)
+            check()
+            row.update(linear_graph_us=round(tgr, 2), linear_graph_tflops=tf(fl, tgr))
+            del graph
+        except Exception as exc:  # report, keep the rest of the table
+            row["graph_error"] = str(exc)[:200]
+        emit(row)
+
+    # configs 1, 2, 4: independent linears
+    for cfg in (1, 2, 4):
+        for case in config_cases(cfg):
+            pk = prepare(case)
+            X = dev_bf16(case.x)
+            qa, ws, Y, qi, g = linear_row(cfg, case, pk, X)
+            if cfg == 1:
+                graph_row(case, pk, X, qa, ws, Y, qi, g)
+            del pk, X, qa, ws, Y
+            torch.cuda.empty_cache()
+
+    # config 3: MLP block, GELU between, measured amax vs amax from the up-projection's epilogue
+    up, down = config_cases(3)
+    pu, pd = prepare(up), prepare(down)
+    X = dev_bf16(up.x)
+    qa_u, ws_u, H, qi_u, g_u = linear_row(3, up, pu, X, epi=1)
+    M = up.M
+    ws_d = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, down.K, down.r), dev)
+    qa_d = w4.quantize_act(H, pd.inv_s, pd.L1t, pd.t_w, workspace=ws_d)
+    Yd = torch.empty(M, down.N, dtype=torch.bfloat16, device=dev)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+
+    def qd():
+        w4.nvfp4_quantize_act(H, M, down.K, down.K, pd.inv_s, pd.L1t, down.r, pd.t_w, qa_d.Xq, qa_d.Xsf,
+                              qa_d.t_x, qa_d.U, ws_d, s)
+
+    def qd_given():
+        w4.nvfp4_quantize_act_with_amax(H, M, down.K, down.K, pd.inv_s, pd.L1t, down.r, pd.t_w, amax, qa_d.Xq,
+                                        qa_d.Xsf, qa_d.t_x, qa_d.U, ws_d, s)
+
+    def gd():
+        w4.gemm(qa_d, pd, Y=Yd)
+
+    def up_amax():
+        amax.zero_()
+        w4.gemm(qa_u, pu, epilogue=w4.EPI_GELU_TANH, Y=H, next_inv_s=pd.inv_s, next_amax=amax)
+
+    tq, tg = med_us([qd, gd])
+    fl_d = flops_per_step(M, down.K, down.N, down.r)
+    qbytes = 2 * M * down.K + M * down.K // 2 + M * down.K // 16 + 2 * M * 2 * down.r
+    emit({"table": "linear", "config": 3, "layer": down.name, "M": M, "K": down.K, "N": down.N, "r": down.r,
+          "input": "GELU output of the up-projection",
+          "quant_us": round(tq, 2), "quant_gbs": round(qbytes / (tq * 1e-6) / 1e9, 1),
+          "quant_frac_hbm": round(qbytes / (tq * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+          "gemm_us": round(tg, 2), "gemm_tflops": tf(gemm_flops(M, down.K, down.N, down.r), tg),
+          "gemm_frac_fp4": round(tf(gemm_flops(M, down.K, down.N, down.r), tg) / fp4_peak, 3)})
+    (tb_meas,) = med_us([lambda: (qi_u(), g_u(), qd(), gd())])
+    (tb_fused,) = med_us([lambda: (qi_u(), up_amax(), qd_given(), gd())])
+    (t_ua, t_qg) = med_us([up_amax, qd_given])
+    check()
+    fl_b = flops_per_step(M, up.K, up.N, up.r) + fl_d
+    emit({"table": "mlp_block", "config": 3, "M": M,
+          "block_us_measured_amax": round(tb_meas, 2), "block_tflops_measured_amax": tf(fl_b, tb_meas),
+          "block_us_epilogue_amax": round(tb_fused, 2), "block_tflops_epilogue_amax": tf(fl_b, tb_fused),
+          "gemm_up_with_amax_us": round(t_ua, 2), "quant_down_given_amax_us": round(t_qg, 2)})
+    del pu, pd, X, qa_u, ws_u, H, ws_d, qa_d, Yd
+    torch.cuda.empty_cache()
+
+    # config 5: the denoising block (fused QKV + MLP-up projection on one
+    # quantised activation, GELU on the MLP part, MLP-down) per step, and a
+    # 50-step trajectory; every step re-quantises a fresh activation
+    qkv, mlp, dn = config_cases(5)
+    K = qkv.K
+    w_cat = np.concatenate([qkv.w, mlp.w], axis=0)
+    b_cat = np.concatenate([qkv.bias, mlp.bias])
+    x_cal = np.concatenate([trajectory_step_activation(t, 10, K)[0] for t in range(50)], axis=0)
+    pf = prep.svdquant_prepare(dev_bf16(w_cat), dev_bf16(x_cal), r=32, bias=dev_bf16(b_cat))
+    w_q, w_m = pf.rows(0, qkv.N), pf.rows(qkv.N, w_cat.shape[0])
+    pdn = prepare(dn)
+    del w_cat
+    for B in (1, 2, 4):
+        M = 4608 * B
+        acts = [dev_bf16(np.concatenate([trajectory_step_activation(t, 4608, K)[0]] * B, axis=0))
+                for t in range(3)]
+        ws1 = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, 32), dev)
+        ws2 = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, dn.K, 32), dev)
+        qa1 = w4.quantize_act(acts[0], pf.inv_s, pf.L1t, pf.t_w, workspace=ws1)
+        Yq = torch.empty(M, qkv.N, dtype=torch.bfloat16, device=dev)
+        Hm = torch.empty(M, mlp.N, dtype=torch.bfloat16, device=dev)
+        qa2 = w4.quantize_act(Hm, pdn.inv_s, pdn.L1t, pdn.t_w, workspace=ws2)
+        Yd = torch.empty(M, dn.N, dtype=torch.bfloat16, device=dev)
+
+        def block(t=0):
+            Xs = acts[t % 3]
+            w4.nvfp4_quantize_act(Xs, M, K, K, pf.inv_s, pf.L1t, 32, pf.t_w, qa1.Xq, qa1.Xsf, qa1.t_x, qa1.U,
+                                  ws1, s)
+            w4.gemm(qa1, w_q, Y=Yq)
+            w4.gemm(qa1, w_m, epilogue=w4.EPI_GELU_TANH, Y=Hm)
+            w4.nvfp4_quantize_act(Hm, M, dn.K, dn.K, pdn.inv_s, pdn.L1t, 32, pdn.t_w, qa2.Xq, qa2.Xsf, qa2.t_x,
+                                  qa2.U, ws2, s)
+            w4.gemm(qa2, pdn, Y=Yd)
+
+        (t_step,) = med_us([block])
+        for t in range(3):
+            block(t)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for t in range(50):
+            block(t)
+        e1.record(s)
+        torch.cuda.synchronize()
+        t_traj = e0.elapsed_time(e1)
+        check()
+        fl = (flops_per_step(M, K, qkv.N, 32) + flops_per_step(M, K, mlp.N, 32)
+              + flops_per_step(M, dn.K, dn.N, 32))
+        emit({"table": "denoising_block", "config": 5, "batch": B, "M": M,
+              "step_us_l2_flushed": round(t_step, 2), "step_tflops": tf(fl, t_step),
+              "trajectory_50_steps_ms": round(t_traj, 3), "trajectory_tflops": tf(50 * fl, t_traj * 1e3),
+              "trajectory_note": "50 steps back to back, three rotating activations, no L2 flush"})
+        del acts, ws1, ws2, qa1, qa2, Yq, Hm, Yd
+        torch.cuda.empty_cache()
 
 
 # ---------------------------------------------------------------- oracle arms
@@ -408,10 +676,15 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=256)
     ap.add_argument("--ref-cols", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table", action="store_true",
+                    help="time every configuration's layers (one JSON line per row) instead of the benchmark step")
+    ap.add_argument("--table-reps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.table:
+        run_table(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -20,6 +20,7 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_pack_weight", "w4a4_gemm", "w4a4_linear", "w4a4_device_status",
     "w4a4_status_string", "EPI_NONE", "EPI_GELU_TANH", "SRC_BF16", "SRC_F32",
     "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
+    "new_workspace",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -167,6 +168,12 @@ def _u8(n, device):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
+def new_workspace(nbytes, device):
+    """A workspace for the entry points that take one: zeroed once, as the
+    library's counters must start at zero (every call leaves them zero)."""
+    return torch.zeros(max(16, nbytes), dtype=torch.uint8, device=device)
+
+
 class QuantizedActivation:
     """Outputs of nvfp4_quantize_act: codes, SF atoms, tensor scale, low-rank U."""
 
@@ -198,9 +205,13 @@ class PackedWeight:
                             None if self.bias is None else self.bias[r0:r1])
 
 
-def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None, amax=None) -> QuantizedActivation:
+def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None, amax=None,
+                 workspace=None) -> QuantizedActivation:
     """NVFP4 activation quantisation; ``amax`` (fp32 device scalar, e.g. from
-    ``gemm(..., next_amax=...)``) supplies the tensor amax instead of measuring it."""
+    ``gemm(..., next_amax=...)``) supplies the tensor amax instead of measuring it.
+    ``workspace``: a uint8 device tensor from ``new_workspace`` of at least
+    ``nvfp4_quant_workspace_bytes(M, K, r)`` bytes, reused across calls (a
+    fresh one is made when None)."""
     M, K = X.shape
     r = 0 if L1t is None else int(L1t.shape[0])
     dev = X.device
@@ -208,7 +219,7 @@ def quantize_act(X: torch.Tensor, inv_s=None, L1t=None, t_w=None, stream=None, a
     Xsf = _u8(nvfp4_sf_bytes(M, K), dev)
     t_x = torch.empty(1, dtype=torch.float32, device=dev)
     U = torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev) if r else None
-    ws = _u8(max(16, nvfp4_quant_workspace_bytes(M, K, r)), dev)
+    ws = new_workspace(nvfp4_quant_workspace_bytes(M, K, r), dev) if workspace is None else workspace
     if amax is None:
         nvfp4_quantize_act(X, M, K, X.stride(0), inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, ws, stream)
     else:
@@ -223,7 +234,7 @@ def pack_weight(R: torch.Tensor, inv_s=None, L1t=None, L2t=None, bias=None, stre
     Wq = _u8(N * K // 2, dev).view(N, K // 2)
     Wsf = _u8(nvfp4_sf_bytes(N, K), dev)
     t_w = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = _u8(max(16, nvfp4_quant_workspace_bytes(N, K, 0)), dev)
+    ws = new_workspace(nvfp4_quant_workspace_bytes(N, K, 0), dev)
     nvfp4_pack_weight(R, src, N, K, R.stride(0), Wq, Wsf, t_w, ws, stream)
     return PackedWeight(Wq, Wsf, t_w, N, K, inv_s, L1t, L2t, bias)
 
@@ -249,7 +260,7 @@ def linear(X: torch.Tensor, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, w
     if Y is None:
         Y = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
     if workspace is None:
-        workspace = _u8(max(16, w4a4_workspace_bytes(M, w.N, K, w.r)), X.device)
+        workspace = new_workspace(w4a4_workspace_bytes(M, w.N, K, w.r), X.device)
     w4a4_linear(X, M, w.N, K, w.Wq, w.Wsf, w.t_w, w.inv_s, w.L1t, w.L2t, w.r, w.bias, epilogue, Y,
                 workspace, stream)
     return Y

@@ -109,20 +109,29 @@ struct GemmCfg {
   static_assert(HALF % 32 == 0, "epilogue column split");
 };
 
-// GELU, tanh form: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715 y^3),
-// with the hardware tanh (tanh.approx.f32, relative error about 2^-11, far
-// inside the bf16 rounding of the result).  No division: the earlier
-// y / (1 + exp(-2u)) form took the IEEE division's slow path whenever exp
-// overflowed (large negative y), which made the epilogue the bottleneck.
-__device__ __forceinline__ float tanh_approx(float x) {
+// GELU, tanh form: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715 y^3).
+// With t = exp(-2|u|) in (0, 1] the same value is y / (1 + t) for y >= 0 and
+// y t / (1 + t) for y < 0: no cancellation on either side (1 + tanh(u) for
+// large negative y would lose all its digits), no overflow (t underflows to 0
+// for large |y|, giving y and -0), and no IEEE division (its slow path made
+// the epilogue the bottleneck).  The hardware base-2 exponential and
+// reciprocal keep the result within a few fp32 ulps, far inside the bf16
+// rounding of the output.
+__device__ __forceinline__ float ex2_approx(float x) {
   float r;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
 __device__ __forceinline__ float gelu_tanh_f32(float y) {
   const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
-  const float hy = 0.5f * y;
-  return fmaf(hy, tanh_approx(u), hy);
+  const float t = ex2_approx(-2.8853900817779268f * fabsf(u));  // exp(-2|u|) = 2^(-2 log2(e) |u|)
+  const float num = y < 0.0f ? y * t : y;
+  return num * rcp_approx(1.0f + t);
 }
 
 template <class C>
@@ -176,6 +185,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the tail of the previous kernel in the stream
+  // (programmatic launch); nothing below may touch memory before this
+  grid_dependency_wait();
 
   const int m_tiles = (p.M + C::BM - 1) / C::BM;
   const int n_tiles = (p.N + BN - 1) / BN;

@@ -160,6 +160,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   cluster_sync();  // both CTAs' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the tail of the previous kernel in the stream
+  // (programmatic launch); nothing below may touch memory before this
+  grid_dependency_wait();
 
   const int m_tiles = (p.M + 2 * C::BM - 1) / (2 * C::BM);
   const int n_tiles = (p.N + BN - 1) / BN;

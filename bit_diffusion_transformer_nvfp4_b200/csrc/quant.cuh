@@ -3,8 +3,7 @@
 //   amax_kernel   pass 1: A = max |x * inv_s| over the tensor.  Grid-stride,
 //                 16-byte loads, warp-shuffle + shared-memory block max, one
 //                 partial maximum per CTA (no atomics, so the result is
-//                 deterministic).  Also clears the per-row-block tickets that
-//                 pass 2 uses.
+//                 deterministic).
 //   quant_kernel  pass 2: one CTA per (128-row block, K slice).  TMA streams
 //                 128 x 64 tiles of the source through a 4-stage mbarrier
 //                 ring (128-byte swizzle); thread t owns row t of the tile,
@@ -17,6 +16,11 @@
 //                 partial, and the last slice of a row block (ticket counter)
 //                 sums the partials in slice order, scales by 1/(t_x t_w) and
 //                 writes the bf16 hi/lo pair.
+//
+// Counters in the workspace (grid barrier, tensor amax word, per-row-block
+// tickets) are zero at rest: every kernel that uses one returns it to zero
+// before it ends (the last participant to read it clears it), so a call needs
+// no memset as long as the workspace was zeroed once before its first use.
 //
 // The quantiser follows the NVFP4 arithmetic stated in include/w4a4.h; every
 // rounding step is an explicit correctly rounded fp32 intrinsic so that codes
@@ -31,15 +35,18 @@ constexpr int kAmaxThreads = 256;
 constexpr int kAmaxMaxBlocks = 1024;
 constexpr int kQRows = 128;       // rows per CTA (one TMEM lane per row)
 constexpr int kQChunk = 64;       // K elements per pipeline step (one SF atom column)
-// Two-pass quantiser (pass 2): three groups of four compute warps (one thread
-// per row of the 128-row tile, group g takes chunks g, g+3, ...), a TMA
-// producer warp and the TMEM owner / U-MMA warp; one CTA per SM.
+// Streaming quantiser (pass 2), persistent, one CTA per SM: three groups of
+// four compute warps (one thread per row of the 128-row tile; group g takes
+// the CTA's chunks g, g+3, ...), a TMA producer warp, the TMEM owner / U-MMA
+// warp and four U warps (one per TMEM lane quarter).
 constexpr int kQGroups = 3;
 constexpr int kQComputeWarps = 4 * kQGroups;
 constexpr int kQProducerWarp = kQComputeWarps;      // TMA producer
 constexpr int kQMmaWarp = kQComputeWarps + 1;       // TMEM owner, issues the U = X L1 MMAs
-constexpr int kQThreads = 32 * (kQComputeWarps + 2);
-constexpr int kQTargetCtas = 592;  // about four work items per SM on a 148-SM part
+constexpr int kQUWarp0 = kQComputeWarps + 2;        // four warps: partial U out, row-block sums
+constexpr int kQThreads = 32 * (kQComputeWarps + 6);
+constexpr int kQMaxSplits = 32;   // K slices per row block at most (each adds a partial U to sum)
+constexpr int kQAcc = 4;          // U accumulators in TMEM: the MMAs run up to three items ahead of the U warps
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -63,8 +70,7 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restri
                                                             int64_t K, int64_t ld,
                                                             const float* __restrict__ inv_s,
                                                             float* __restrict__ partials,
-                                                            int* __restrict__ tickets,
-                                                            int n_tickets, int rows_per_cta) {
+                                                            int rows_per_cta) {
   constexpr int EPV = 16 / sizeof(SrcT);  // channels per 16-byte segment
   const int lane = threadIdx.x & 31;
   const int64_t segs = K / EPV;
@@ -127,9 +133,6 @@ __global__ void __launch_bounds__(kAmaxThreads) amax_kernel(const SrcT* __restri
     r = warp_max(r);
     if (threadIdx.x == 0) partials[cta] = r;
   }
-  if (cta == 0) {
-    for (int t = threadIdx.x; t < n_tickets; t += blockDim.x) tickets[t] = 0;
-  }
 }
 
 // ------------------------------------------------------------------ pass 2
@@ -157,17 +160,21 @@ struct QuantTile {
   // bf16: one 128 x 64 box (16 KB); fp32: two 128 x 32 boxes (32 KB).
   static constexpr int kBytes = kQRows * kQChunk * static_cast<int>(sizeof(SrcT));
   static constexpr int kBoxes = sizeof(SrcT) / 2;
-  static constexpr int kStages = sizeof(SrcT) == 2 ? 10 : 6;
+  static constexpr int kStages = sizeof(SrcT) == 2 ? 9 : 6;
   static constexpr int kL1Bytes = 32 * kQChunk * 2;  // L1t tile, 32 x 64 bf16 (4 KB)
   static constexpr int kL1Off = kBytes;
   static constexpr int kInvSOff = kBytes + (sizeof(SrcT) == 2 ? kL1Bytes : 0);  // 64 fp32 of inv_s
   static constexpr int kStageBytes = (kInvSOff + kQChunk * 4 + 1023) / 1024 * 1024;
-  // ring, 1 KB alignment slack, barriers + scalars (512 B), the 256-entry
-  // table of code multipliers
-  static constexpr int kBarOff = kStageBytes * kStages;
-  static constexpr int kRqOff = kBarOff + 512;
-  static constexpr int kSmem = kRqOff + 1024 + 1024;
-  static_assert(8 * (3 * kStages + 1) + 4 * (2 + kQThreads / 32 + 1) <= 512, "barrier area");
+  // ring, then per compute warp two 1 KB staging buffers for its codes (32
+  // rows x 32 bytes, written out by TMA), barriers + scalars (512 B), 1 KB
+  // alignment slack
+  static constexpr int kCodeBuf = 32 * 32;
+  static constexpr int kCodeOff = kStageBytes * kStages;
+  static constexpr int kBarOff = kCodeOff + kQComputeWarps * 2 * kCodeBuf;
+  static constexpr int kSmem = kBarOff + 512 + 1024;
+  // full/empty/mma_done per stage, acc_full/acc_empty per accumulator, drain;
+  // then the TMEM address, abort flag, per-warp maxima and the last-slice flag
+  static_assert(8 * (3 * kStages + 2 * kQAcc + 1) + 4 * (2 + kQThreads / 32 + 1) <= 512, "barrier area");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -228,60 +235,84 @@ __device__ __forceinline__ float tensor_scale_from(float amax) {
 }
 
 // The last K slice of a row block sums the fp32 partials in slice order,
-// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row.
+// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row (columns in
+// two halves of 16, two slices' loads in flight).
 __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, int64_t rows_pad, int64_t prow,
                                                  int64_t row) {
   __threadfence();
-  float acc[32];
+  const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
+    float acc[16];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
-  for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
-    // the loads of two slices are in flight together; the sums still run in
-    // slice order
-    float4 w[2][8];
+    for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+    for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
+      float4 w[2][4];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (sp0 + q < p.splits) {
-        const float4* src =
-            reinterpret_cast<const float4*>(p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow) * 32);
+      for (int q = 0; q < 2; ++q) {
+        if (sp0 + q < p.splits) {
+          const float4* src = reinterpret_cast<const float4*>(
+              p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow) * 32 + 16 * hh);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[q][j] = __ldcg(src + j);
+          for (int j = 0; j < 4; ++j) w[q][j] = __ldcg(src + j);
+        }
       }
-    }
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (sp0 + q < p.splits) {
+      for (int q = 0; q < 2; ++q) {
+        if (sp0 + q < p.splits) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          acc[4 * j] = __fadd_rn(acc[4 * j], w[q][j].x);
-          acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], w[q][j].y);
-          acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], w[q][j].z);
-          acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], w[q][j].w);
+          for (int j = 0; j < 4; ++j) {
+            acc[4 * j] = __fadd_rn(acc[4 * j], w[q][j].x);
+            acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], w[q][j].y);
+            acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], w[q][j].z);
+            acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], w[q][j].w);
+          }
         }
       }
     }
-  }
-  if (row < p.M) {
-    const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
-    uint32_t hi[16], lo[16];
+    if (row < p.M) {
+      uint32_t hi[8], lo[8];
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-      const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
-      const uint32_t h = pack_bf16x2(a0, a1);
-      hi[j / 2] = h;
-      lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
+      for (int j = 0; j < 16; j += 2) {
+        const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
+        const uint32_t h = pack_bf16x2(a0, a1);
+        hi[j / 2] = h;
+        lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.u_out + row * 64 + 16 * hh);
+      dst[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      dst[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+      dst[4] = make_uint4(lo[0], lo[1], lo[2], lo[3]);  // the lo half starts 32 columns on
+      dst[5] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
     }
-    uint4* dst2 = reinterpret_cast<uint4*>(p.u_out + row * 64);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) dst2[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) dst2[4 + j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
   }
+}
+
+// Division by 6 of a non-negative fp32 value, correctly rounded for every
+// input >= 2^-100 (Markstein's correction: one residual step from the
+// rounded reciprocal, P. Markstein, IBM J. Res. Develop. 34(1), 1990; checked
+// against IEEE division on every float from 2^-100 up).  Block maxima below
+// 2^-100 give a zero E4M3 scale either way.
+__device__ __forceinline__ float div6(float x) {
+  const float c = 0.16666667f;  // RN(1/6)
+  const float q0 = __fmul_rn(x, c);
+  return __fmaf_rn(__fmaf_rn(-6.0f, q0, x), c, q0);
+}
+
+// max |v[j]| over 16 values, as a tree (four dependent steps).
+__device__ __forceinline__ float absmax16(const float* v) {
+  float m[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m[j] = fmaxf(fabsf(v[j]), fabsf(v[j + 8]));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m[j] = fmaxf(m[j], m[j + 4]);
+  return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
 }
 
 template <typename SrcT>
 __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                           const __grid_constant__ CUtensorMap tm_l1,
+                                                          const __grid_constant__ CUtensorMap tm_q,
                                                           const QuantParams p) {
   using Tile = QuantTile<SrcT>;
   constexpr int S = Tile::kStages;
@@ -290,23 +321,24 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tile::kBarOff);
   uint64_t* empty = full + S;
   uint64_t* mma_done = empty + S;
-  uint64_t* drain = mma_done + S;
+  uint64_t* acc_full = mma_done + S;              // [kQAcc] an item's U MMAs are complete
+  uint64_t* acc_empty = acc_full + kQAcc;         // [kQAcc] the U warps have read the accumulator
+  uint64_t* drain = acc_empty + kQAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(tmem_slot + 2);  // one float per warp
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 2 + kQThreads / 32);
-  float* rq_tab = reinterpret_cast<float*>(smem + Tile::kRqOff);  // 1/(dec(e) t) per scale code
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2 + kQThreads / 32);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int rb = blockIdx.x;
-  const int split = blockIdx.y;
   const int chunks = static_cast<int>(p.K / kQChunk);
-  const int kc0 = split * p.chunks_per_split;
-  const int kc1 = min(kc0 + p.chunks_per_split, chunks);
-  const int n = kc1 - kc0;
+  const int n_items = p.row_blocks * p.splits;
   const bool lr = p.has_lr != 0;
+  grid_launch_dependents();
+
+  // Work item w: row block w / splits, chunks [split * cps, ...) of its K.
+  auto item_chunks = [&](int w) { return min(p.chunks_per_split, chunks - (w % p.splits) * p.chunks_per_split); };
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -314,12 +346,16 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       mbar_init(smem_u32(&empty[s]), 4);  // the four warps of the group that took the chunk
       mbar_init(smem_u32(&mma_done[s]), 1);
     }
+    for (int a = 0; a < kQAcc; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), 4);  // the four U warps
+    }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (lr && warp == kQMmaWarp) {
-    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_alloc(smem_u32(tmem_slot), 32 * kQAcc);  // 32-column U accumulators
     tmem_relinquish();
   }
   // tensor scale from the pass-1 partial maxima (the same value in every CTA)
@@ -335,7 +371,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
   for (int w = 1; w < kQThreads / 32; ++w) amax = fmaxf(amax, red[w]);
   const float t = tensor_scale_from(amax);
   const float rt = __frcp_rn(t);
-  if (rb == 0 && split == 0 && tid == 0) *p.t_out = t;
+  if (blockIdx.x == 0 && tid == 0) *p.t_out = t;
   const uint32_t tmem = lr ? *tmem_slot : 0u;
 
   if (warp == kQProducerWarp) {
@@ -343,73 +379,142 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
     if (lane == 0) {
       tma_prefetch_desc(&tm_x);
       if (lr) tma_prefetch_desc(&tm_l1);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int s = i % S;
-        if (i >= S) {
-          const uint32_t ph = ((i / S) - 1) & 1;   // the fill of chunk i - S
-          if (!mbar_wait(smem_u32(&empty[s]), ph, abort_flag, p.status)) break;
-          if (lr && !mbar_wait(smem_u32(&mma_done[s]), ph, abort_flag, p.status)) break;
+      const uint32_t inv_bytes = p.inv_s != nullptr ? kQChunk * 4 : 0;
+      int c = 0;  // this CTA's chunks, in order
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        const int rb = w / p.splits;
+        const int kc0 = (w % p.splits) * p.chunks_per_split;
+        const int n = item_chunks(w);
+        for (int i = 0; i < n; ++i, ++c) {
+          const int s = c % S;
+          if (c >= S) {
+            const uint32_t ph = ((c / S) - 1) & 1;  // the fill of chunk c - S
+            if (!mbar_wait(smem_u32(&empty[s]), ph, abort_flag, p.status) ||
+                (lr && !mbar_wait(smem_u32(&mma_done[s]), ph, abort_flag, p.status))) {
+              ok = false;
+              break;
+            }
+          }
+          const uint32_t bar = smem_u32(&full[s]);
+          uint8_t* dst = smem + s * Tile::kStageBytes;
+          const int kx = (kc0 + i) * kQChunk;
+          if constexpr (sizeof(SrcT) == 2) {
+            mbar_arrive_expect_tx(bar, Tile::kBytes + (lr ? Tile::kL1Bytes : 0) + inv_bytes);
+            tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
+            if (lr) tma_load_2d(smem_u32(dst + Tile::kL1Off), &tm_l1, bar, kx, 0);
+          } else {
+            mbar_arrive_expect_tx(bar, Tile::kBytes + inv_bytes);
+            tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
+            tma_load_2d(smem_u32(dst + kQRows * 128), &tm_x, bar, kx + 32, rb * kQRows);
+          }
+          if (inv_bytes) bulk_load(smem_u32(dst + Tile::kInvSOff), p.inv_s + kx, inv_bytes, bar);
         }
-        const uint32_t bar = smem_u32(&full[s]);
-        uint8_t* dst = smem + s * Tile::kStageBytes;
-        const int kx = (kc0 + i) * kQChunk;
-        const uint32_t inv_bytes = p.inv_s != nullptr ? kQChunk * 4 : 0;
-        if constexpr (sizeof(SrcT) == 2) {
-          mbar_arrive_expect_tx(bar, Tile::kBytes + (lr ? Tile::kL1Bytes : 0) + inv_bytes);
-          tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
-          if (lr) tma_load_2d(smem_u32(dst + Tile::kL1Off), &tm_l1, bar, kx, 0);
-        } else {
-          mbar_arrive_expect_tx(bar, Tile::kBytes + inv_bytes);
-          tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
-          tma_load_2d(smem_u32(dst + kQRows * 128), &tm_x, bar, kx + 32, rb * kQRows);
-        }
-        if (inv_bytes) bulk_load(smem_u32(dst + Tile::kInvSOff), p.inv_s + kx, inv_bytes, bar);
-        ++issued;
       }
       // every fill issued must land before the shared memory is released
-      for (int j = max(0, issued - S); j < issued; ++j) mbar_wait_drain(smem_u32(&full[j % S]), (j / S) & 1);
+      for (int j = max(0, c - S); j < c; ++j) mbar_wait_drain(smem_u32(&full[j % S]), (j / S) & 1);
     }
   } else if (warp == kQMmaWarp) {
-    // ------------------------------------------------------- U = X L1 MMAs
+    // ------------------------------------------------------- U = X L1 MMAs, one accumulator per item
     if (lr && lane == 0) {
-      for (int i = 0; i < n; ++i) {
-        const int s = i % S;
-        if (!mbar_wait(smem_u32(&full[s]), (i / S) & 1, abort_flag, p.status)) break;
+      int c = 0, j = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++j) {
+        const int a = j % kQAcc;
+        if (j >= kQAcc && !mbar_wait(smem_u32(&acc_empty[a]), ((j / kQAcc) - 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * Tile::kStageBytes);
-        const uint32_t b_base = a_base + Tile::kL1Off;
+        const uint32_t d = tmem + 32u * a;
+        const int n = item_chunks(w);
+        for (int i = 0; i < n; ++i, ++c) {
+          const int s = c % S;
+          if (!mbar_wait(smem_u32(&full[s]), (c / S) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * Tile::kStageBytes);
+          const uint32_t b_base = a_base + Tile::kL1Off;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
-          mma_bf16(tmem, ad, bd, idesc_bf16(128, 32), (i > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
+            mma_bf16(d, ad, bd, idesc_bf16(128, 32), (i > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&mma_done[s]));
         }
-        tc_commit(smem_u32(&mma_done[s]));
+        if (ok) tc_commit(smem_u32(&acc_full[a]));
       }
-      // all MMAs of this thread complete before TMEM is read or released
+      // all MMAs of this thread complete before TMEM is released
       tc_commit(smem_u32(drain));
       mbar_wait_drain(smem_u32(drain), 0);
     }
+  } else if (warp >= kQUWarp0) {
+    // ------------------------------------------------------- partial U out; row-block sums
+    if (lr) {
+      const int quarter = warp & 3;  // the TMEM lane quarter this warp may read
+      const int ut = (warp - kQUWarp0) * 32 + lane;
+      const int64_t rows_pad = static_cast<int64_t>(p.row_blocks) * kQRows;
+      int j = 0;
+      for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++j) {
+        const int a = j % kQAcc;
+        const int rb = w / p.splits;
+        const int split = w % p.splits;
+        if (!mbar_wait(smem_u32(&acc_full[a]), (j / kQAcc) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        uint32_t u[32];
+        tmem_ld_32cols(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 32u * a, u);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&acc_empty[a]));
+        const int64_t prow = static_cast<int64_t>(rb) * kQRows + quarter * 32 + lane;
+        float4* dst = reinterpret_cast<float4*>(p.u_part + (static_cast<int64_t>(split) * rows_pad + prow) * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                               __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+        __threadfence();
+        named_bar_sync(2, 128);  // the four U warps' partial rows are out
+        if (ut == 0) {
+          const int ticket = atomicAdd(&p.tickets[rb], 1);
+          const bool last = ticket == p.splits - 1;
+          if (last) p.tickets[rb] = 0;  // every slice has taken its ticket
+          *last_flag = last ? 1 : 0;
+        }
+        named_bar_sync(2, 128);
+        if (*last_flag) {
+          // this was the row block's last slice: sum every slice's partial
+          // for row ut of the block, in slice order
+          const int64_t frow = static_cast<int64_t>(rb) * kQRows + ut;
+          finalize_lowrank(p, t, rows_pad, frow, frow);
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------- quantise rows
-    // The code multiplier of every scale code, once per CTA (the same
-    // __frcp_rn(dec(e) * t) as a per-block computation).
     const bool has_inv = p.inv_s != nullptr;
-    for (int e = tid; e < 256; e += 32 * kQComputeWarps)
-      rq_tab[e] = __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(e)).y, t));
-    named_bar_sync(1, 32 * kQComputeWarps);
+    if (lane == 0) tma_prefetch_desc(&tm_q);
+    // this warp's 32 rows of codes go out through two staging buffers
+    uint8_t* code_stage = smem + Tile::kCodeOff + warp * 2 * Tile::kCodeBuf;
+    int n_stored = 0;
     const int grp = warp >> 2;
     const int row_in_tile = tid & (kQRows - 1);
-    const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-    const bool row_ok = row < p.M;
-    const int64_t kbytes = p.K / 2;
-    for (int i = grp; i < n; i += kQGroups) {
-      const int s = i % S;
-      if (!mbar_wait(smem_u32(&full[s]), (i / S) & 1, abort_flag, p.status)) break;
+    int w = blockIdx.x;   // the item that holds chunk c
+    int item_c0 = 0;      // its first chunk (this CTA's count)
+    int item_n = w < n_items ? item_chunks(w) : 0;
+    for (int c = grp; w < n_items; c += kQGroups) {
+      while (w < n_items && c >= item_c0 + item_n) {
+        item_c0 += item_n;
+        w += gridDim.x;
+        item_n = w < n_items ? item_chunks(w) : 0;
+      }
+      if (w >= n_items) break;
+      const int rb = w / p.splits;
+      const int kc = (w % p.splits) * p.chunks_per_split + (c - item_c0);
+      const int s = c % S;
+      if (!mbar_wait(smem_u32(&full[s]), (c / S) & 1, abort_flag, p.status)) break;
       const uint8_t* tile = smem + s * Tile::kStageBytes;
       const float* inv = reinterpret_cast<const float*>(tile + Tile::kInvSOff);
-      const int kc = kc0 + i;
       uint32_t cw[8];
       uint32_t e4 = 0u;
 #pragma unroll
@@ -419,27 +524,22 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           load_unit<SrcT>(tile, inv, has_inv, row_in_tile, 4 * h + u, *reinterpret_cast<float(*)[8]>(&x[8 * u]));
-        float bm0 = 0.0f, bm1 = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          bm0 = fmaxf(bm0, fabsf(x[j]));
-          bm1 = fmaxf(bm1, fabsf(x[16 + j]));
-        }
+        const float bm0 = absmax16(x), bm1 = absmax16(x + 16);
         // both blocks' scale bytes in one conversion; byte 0 = block 2h
-        const uint32_t e2 = cvt_e4m3x2(__fdiv_rn(__fmul_rn(bm1, rt), 6.0f), __fdiv_rn(__fmul_rn(bm0, rt), 6.0f)) & 0xFFFFu;
+        const uint32_t e2 = cvt_e4m3x2(div6(__fmul_rn(bm1, rt)), div6(__fmul_rn(bm0, rt))) & 0xFFFFu;
         e4 |= e2 << (16 * h);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const uint32_t e = (e2 >> (8 * q)) & 0xFFu;
           cw[4 * h + 2 * q] = cw[4 * h + 2 * q + 1] = 0u;
           if (e != 0u) {  // a zero scale leaves the block's codes +0
-            const float rq = rq_tab[e];
+            const float rq = __frcp_rn(__fmul_rn(e4m3x2_to_f32(e).y, t));  // 1/(dec(e) t)
 #pragma unroll
             for (int uu = 0; uu < 2; ++uu) {
               float v[8];
 #pragma unroll
-              for (int j = 0; j < 8; j += 2)
-                mul2_rn(v[j], v[j + 1], x[16 * q + 8 * uu + j], x[16 * q + 8 * uu + j + 1], rq, rq);
+              for (int jj = 0; jj < 8; jj += 2)
+                mul2_rn(v[jj], v[jj + 1], x[16 * q + 8 * uu + jj], x[16 * q + 8 * uu + jj + 1], rq, rq);
               cw[4 * h + 2 * q + uu] = cvt_e2m1x8(v);
             }
           }
@@ -451,63 +551,41 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-      if (row_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(p.q + row * kbytes + static_cast<int64_t>(kc) * 32);
-        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      // codes: row ``lane`` of the warp's 32 rows, 32 bytes, into a staging
+      // buffer the TMA store of two chunks ago has finished reading; lanes
+      // with bit 2 set store their halves in the other order (no bank
+      // conflicts); the TMA store drops rows >= M
+      uint8_t* cb = code_stage + (n_stored & 1) * Tile::kCodeBuf;
+      if (n_stored >= 2) {
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
       }
+      const int first = (lane >> 2) & 1;
+      *reinterpret_cast<uint4*>(cb + lane * 32 + 16 * first) =
+          first ? make_uint4(cw[4], cw[5], cw[6], cw[7]) : make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      *reinterpret_cast<uint4*>(cb + lane * 32 + 16 * (first ^ 1)) =
+          first ? make_uint4(cw[0], cw[1], cw[2], cw[3]) : make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tm_q, smem_u32(cb), kc * 32, rb * kQRows + (warp & 3) * 32);
+        bulk_commit_group();
+      }
+      ++n_stored;
       const int64_t atom = static_cast<int64_t>(rb) * chunks + kc;
       *reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (row_in_tile & 31) * 16 + (row_in_tile >> 5) * 4) = e4;
     }
+    // the code stores have landed before the CTA ends
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   // Every role has finished (or given up); in-flight copies and MMAs drained.
   tc_fence_before();
   __syncthreads();
-  const bool aborted = *abort_flag != 0;
-  if (!lr || aborted) {
-    if (lr && warp == kQMmaWarp) {
-      tc_fence_after();
-      tmem_dealloc(tmem, 32);
-    }
-    return;
-  }
-
-  // U partial of this K slice (TMEM lane = row): warps 0-3 (one per TMEM lane
-  // quarter) read it out.
-  const int row_in_tile = tid;
-  const int64_t rows_pad = static_cast<int64_t>(gridDim.x) * kQRows;
-  const int64_t prow = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-  if (warp < 4) {
+  if (lr && warp == kQMmaWarp) {
     tc_fence_after();
-    uint32_t u[32];
-    tmem_ld_32cols(tmem + (static_cast<uint32_t>(warp * 32) << 16), u);
-    tmem_ld_wait();
-    if (n == 0) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) u[j] = 0u;
-    }
-    float4* dst = reinterpret_cast<float4*>(p.u_part + (static_cast<int64_t>(split) * rows_pad + prow) * 32);
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      dst[j] = make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
-                           __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
-    __threadfence();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kQMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 32);
-  }
-  if (tid == 0) {
-    const int ticket = atomicAdd(&p.tickets[rb], 1);
-    *last_flag = (ticket == p.splits - 1) ? 1 : 0;
-  }
-  __syncthreads();
-  if (*last_flag && warp < 4) {
-    const int64_t row = static_cast<int64_t>(rb) * kQRows + row_in_tile;
-    finalize_lowrank(p, t, rows_pad, prow, row);
+    tmem_dealloc(tmem, 32 * kQAcc);
   }
 }
 
@@ -551,16 +629,6 @@ static_assert(kFComputeWarps * 32 >= 256, "one thread per scale code fills the m
 
 static_assert(kFUWarp0 % 4 == 0 && kFThreads == 32 * (kFUWarp0 + 4), "lane quarters");
 
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // Bounded spin until a global counter reaches ``target``; false on timeout
 // (then the abort flag and the device status are set).
 __device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target, volatile int* abort, int* status) {
@@ -594,9 +662,14 @@ __global__ void __launch_bounds__(kFThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(tmem_slot + 2);  // kFComputeWarps floats
   float* t_shared = reinterpret_cast<float*>(tmem_slot + 2 + kFComputeWarps);
-  unsigned* counter = grid_sync;       // CTAs that have contributed
+  // Zero at rest.  counter: CTAs that have contributed their maximum (first
+  // gridDim.x increments), then CTAs that have read the result (second
+  // gridDim.x); the last reader clears it and the amax word.  tickets[rb]:
+  // slices of the row block whose partial U is out, then slices that have
+  // seen them all; the last clears it.
+  unsigned* counter = grid_sync;
   unsigned* amax_bits = grid_sync + 1; // running max of the CTA maxima (non-negative floats order as bits)
-  unsigned* tickets = grid_sync + 2;   // per row block: slices whose partial U is out
+  unsigned* tickets = grid_sync + 2;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -610,6 +683,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   const bool lr = p.has_lr != 0;
   const bool has_inv = p.inv_s != nullptr;
   const int64_t rows_pad = static_cast<int64_t>(p.row_blocks) * kQRows;
+  grid_launch_dependents();  // all CTAs are resident (cooperative launch)
 
   if (tid == 0) {
     for (int c = 0; c < kFusedMaxChunks; ++c) mbar_init(smem_u32(&full[c]), 1);
@@ -714,7 +788,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // ---------------------------------------------------- wait for the tensor scale
       named_bar_sync(2, kFThreads);
       if (!*abort_flag) {
-        if (tid == 32 * kFUWarp0) spin_until(tickets + rb, static_cast<unsigned>(p.splits), abort_flag, p.status);
+        if (tid == 32 * kFUWarp0 &&
+            spin_until(tickets + rb, static_cast<unsigned>(p.splits), abort_flag, p.status) &&
+            atom_acq_rel_add(tickets + rb, 1u) == 2u * static_cast<unsigned>(p.splits) - 1u)
+          tickets[rb] = 0u;  // every slice has passed
         named_bar_sync(3, 128);
         if (!*abort_flag) {
           // -------------------------------------------------- this CTA's share of the U rows
@@ -785,10 +862,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
         for (int u = 0; u < 8; ++u) {
           float v[8];
           load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, u, v);
-          float bm = bmax[4 * i + u / 2];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) bm = fmaxf(bm, fabsf(v[j]));
-          bmax[4 * i + u / 2] = bm;
+          // |v| maxima as a tree, then into the block's running maximum
+          const float m01 = fmaxf(fabsf(v[0]), fabsf(v[1])), m23 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+          const float m45 = fmaxf(fabsf(v[4]), fabsf(v[5])), m67 = fmaxf(fabsf(v[6]), fabsf(v[7]));
+          bmax[4 * i + u / 2] = fmaxf(bmax[4 * i + u / 2], fmaxf(fmaxf(m01, m23), fmaxf(m45, m67)));
         }
 #pragma unroll
         for (int b = 0; b < 4; ++b) m = fmaxf(m, bmax[4 * i + b]);
@@ -805,10 +882,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
       for (int w = 1; w < kFComputeWarps; ++w) a = fmaxf(a, red[w]);
       atomicMax(amax_bits, __float_as_uint(a));
       red_release_add(counter, 1u);
-      spin_until(counter, gridDim.x, abort_flag, p.status);
-      const float t = tensor_scale_from(__uint_as_float(ld_acquire_gpu(amax_bits)));
-      *t_shared = t;
-      if (blockIdx.x == 0) *p.t_out = t;
+      if (spin_until(counter, gridDim.x, abort_flag, p.status)) {
+        const float t = tensor_scale_from(__uint_as_float(ld_acquire_gpu(amax_bits)));
+        *t_shared = t;
+        if (blockIdx.x == 0) *p.t_out = t;
+        if (atom_acq_rel_add(counter, 1u) == 2u * gridDim.x - 1u) {
+          *amax_bits = 0u;  // every CTA has read it
+          *counter = 0u;
+        }
+      }
     }
     named_bar_sync(1, 32 * kFComputeWarps);
     if (lr) named_bar_arrive(2, kFThreads);  // the tensor scale is out for the U warps
@@ -833,8 +915,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // two blocks' scale bytes in one conversion; byte 0 = block 2h
-          const uint32_t e2 = cvt_e4m3x2(__fdiv_rn(__fmul_rn(bmax[4 * i + 2 * h + 1], rt), 6.0f),
-                                         __fdiv_rn(__fmul_rn(bmax[4 * i + 2 * h], rt), 6.0f)) & 0xFFFFu;
+          const uint32_t e2 = cvt_e4m3x2(div6(__fmul_rn(bmax[4 * i + 2 * h + 1], rt)),
+                                         div6(__fmul_rn(bmax[4 * i + 2 * h], rt))) & 0xFFFFu;
           e4 |= e2 << (16 * h);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -120,24 +121,57 @@ bool encode_sf(CUtensorMap* m, const void* ptr, int64_t rows, int64_t K, uint32_
 struct QuantPlan {
   int64_t row_blocks = 0;
   int chunks = 0, splits = 0, chunks_per_split = 0;
+  int upart_slices = 0;  // K slices the low-rank partial buffer holds
   size_t off_partials = 0, off_tickets = 0, off_upart = 0, bytes = 0;
 };
+
+// SM count the work split and the workspace size assume (B200); on another
+// count the kernels stay correct, only the balance changes.
+constexpr int kPlanSms = 148;
+
+// K-slice count of the single-pass path (its tile set is co-resident: one CTA
+// per (row block, slice), at most kFusedMaxChunks chunks each).
+int fused_splits(int64_t row_blocks, int chunks, int64_t sms) {
+  int64_t want = ceil_div(chunks, kFusedMaxChunks);
+  const int64_t more = row_blocks > 0 ? sms / row_blocks : 1;
+  if (more > want) want = more;
+  if (want > chunks) want = chunks;
+  if (want < 1) want = 1;
+  const int cps = static_cast<int>(ceil_div(chunks, want));
+  return static_cast<int>(ceil_div(chunks, cps));
+}
 
 QuantPlan quant_plan(int64_t M, int64_t K, int r) {
   QuantPlan q;
   q.row_blocks = ceil_div(M, kQRows);
   q.chunks = static_cast<int>(K / kQChunk);
-  int64_t want = q.row_blocks > 0 ? ceil_div(kQTargetCtas, q.row_blocks) : 1;
-  if (want < 1) want = 1;
-  if (want > q.chunks) want = q.chunks;
-  q.chunks_per_split = static_cast<int>(ceil_div(q.chunks, want));
-  q.splits = static_cast<int>(ceil_div(q.chunks, q.chunks_per_split));
+  // Streaming pass: persistent CTAs take the (row block, K slice) items in
+  // turn; pick the slice count whose busiest CTA streams the fewest chunks,
+  // charging four chunks per slice for the partial U it adds to a row block's
+  // sum (ties: fewer slices).
+  q.splits = 1;
+  q.chunks_per_split = q.chunks;
+  int64_t best = -1;
+  for (int sp = 1; sp <= kQMaxSplits && sp <= q.chunks; ++sp) {
+    const int cps = static_cast<int>(ceil_div(q.chunks, sp));
+    const int spl = static_cast<int>(ceil_div(q.chunks, cps));
+    if (spl != sp) continue;
+    const int64_t busiest = ceil_div(q.row_blocks * spl, kPlanSms) * cps + 4 * spl;
+    if (best < 0 || busiest < best) {
+      best = busiest;
+      q.splits = spl;
+      q.chunks_per_split = cps;
+    }
+  }
+  const int slices_max = std::max(q.splits, fused_splits(q.row_blocks, q.chunks, kPlanSms));
   q.off_partials = 0;
   q.off_tickets = round256(sizeof(float) * kAmaxMaxBlocks);
-  // per-row-block tickets, then the single-pass path's grid-barrier counter
-  // and tensor-amax word
+  // counters, zero at rest (each kernel clears what it used): the two-pass
+  // path's per-row-block tickets, or the single-pass path's grid-barrier
+  // counter, tensor-amax word and per-row-block tickets
   q.off_upart = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks + 2));
-  const size_t upart = r > 0 ? sizeof(float) * static_cast<size_t>(q.splits) * q.row_blocks * kQRows * 32 : 0;
+  q.upart_slices = slices_max;
+  const size_t upart = r > 0 ? sizeof(float) * static_cast<size_t>(slices_max) * q.row_blocks * kQRows * 32 : 0;
   q.bytes = q.off_upart + round256(upart);
   return q;
 }
@@ -154,21 +188,14 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   const int64_t rb = plan.row_blocks;
   const int chunks = plan.chunks;
   if (rb < 1 || rb > dev->num_sms) return -1;
-  int64_t want = ceil_div(chunks, kFusedMaxChunks);
-  const int64_t more = dev->num_sms / rb;
-  if (more > want) want = more;
-  if (want > chunks) want = chunks;
-  const int cps = static_cast<int>(ceil_div(chunks, want));
-  const int splits = static_cast<int>(ceil_div(chunks, cps));
-  if (cps > kFusedMaxChunks || rb * splits > dev->num_sms || splits > plan.splits) return -1;
+  const int splits = fused_splits(rb, chunks, dev->num_sms);
+  const int cps = static_cast<int>(ceil_div(chunks, splits));
+  if (cps > kFusedMaxChunks || rb * splits > dev->num_sms || splits > plan.upart_slices) return -1;
 
   uint8_t* w = static_cast<uint8_t*>(ws);
-  // grid-barrier counter, tensor-amax bits, one ticket per row block
+  // grid-barrier counter, tensor-amax bits, one ticket per row block (zero at
+  // rest: the kernel clears them before it ends)
   unsigned* grid_sync = reinterpret_cast<unsigned*>(w + plan.off_tickets);
-  if (cudaMemsetAsync(grid_sync, 0, sizeof(unsigned) * static_cast<size_t>(rb + 2), stream) != cudaSuccess) {
-    cudaGetLastError();
-    return W4A4_ERR_CUDA;
-  }
   CUtensorMap tm_x, tm_l1;
   if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(ld) * 2, 64u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -246,14 +273,8 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   const int64_t grid1 = gx * gy;
   if (amax_in == nullptr) {
     amax_kernel<SrcT><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kAmaxThreads, 0, stream>>>(
-        X, M, K, ld, inv_s, partials, tickets, static_cast<int>(plan.row_blocks), static_cast<int>(rows_per));
+        X, M, K, ld, inv_s, partials, static_cast<int>(rows_per));
     if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
-  } else if (r > 0) {
-    // the amax pass would have zeroed the U tickets
-    if (cudaMemsetAsync(tickets, 0, sizeof(int) * static_cast<size_t>(plan.row_blocks), stream) != cudaSuccess) {
-      cudaGetLastError();
-      return W4A4_ERR_CUDA;
-    }
   }
 
   CUtensorMap tm_x, tm_l1;
@@ -269,6 +290,11 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   } else {
     tm_l1 = tm_x;  // unused
   }
+  // codes, written by TMA: 32 rows x 32 bytes (one 64-wide chunk) per box
+  CUtensorMap tm_q;
+  if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(K / 2), 32u, 32u, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return W4A4_ERR_CUDA;
   QuantParams p;
   p.M = M;
   p.K = K;
@@ -287,8 +313,11 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   p.row_blocks = static_cast<int>(plan.row_blocks);
   p.has_lr = r > 0 ? 1 : 0;
   p.status = dev->status_ptr;
-  const dim3 grid2(static_cast<unsigned>(plan.row_blocks), static_cast<unsigned>(plan.splits));
-  quant_kernel<SrcT><<<grid2, kQThreads, QuantTile<SrcT>::kSmem, stream>>>(tm_x, tm_l1, p);
+  // persistent: one CTA per SM walks the (row block, K slice) work items
+  const int64_t items = plan.row_blocks * plan.splits;
+  const int64_t grid2 = items < dev->num_sms ? items : dev->num_sms;
+  quant_kernel<SrcT><<<static_cast<unsigned>(grid2), kQThreads, QuantTile<SrcT>::kSmem, stream>>>(tm_x, tm_l1, tm_q,
+                                                                                                   p);
   if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
   return W4A4_OK;
 }
@@ -334,8 +363,20 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   p.next_amax = next_amax;
   const int64_t tiles = ceil_div(M, C::BM) * ceil_div(N, C::BN);
   const int64_t grid = tiles < dev->num_sms ? tiles : dev->num_sms;
-  gemm_kernel<C><<<static_cast<unsigned>(grid), C::THREADS, C::SMEM, stream>>>(ta, tb, tsa, tsb, tu, tl, p);
-  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_kernel<C>, ta, tb, tsa, tsb, tu, tl, p) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
   return W4A4_OK;
 }
 
@@ -390,13 +431,15 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, gemm2_kernel<C>, ta, tb, tsa, tsb, tu, tl, ty, p) != cudaSuccess) {
     cudaGetLastError();
     return W4A4_ERR_CUDA;
@@ -595,9 +638,10 @@ namespace {
 void* g_noalloc_ptr[w4a4::kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of g_noalloc_scratch on the current device (set up on the
-// first call per device), or nullptr on failure.
-void* noalloc_scratch() {
+// Device address of g_noalloc_scratch on the current device, or nullptr on
+// failure.  The first call per device also zeroes the array on ``stream``
+// (its counters must start at zero; the kernels leave them zero).
+void* noalloc_scratch(cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= w4a4::kMaxDevices) {
     cudaGetLastError();
@@ -606,7 +650,8 @@ void* noalloc_scratch() {
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (g_noalloc_ptr[dev] == nullptr) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess ||
+        cudaMemsetAsync(ptr, 0, W4A4_NOALLOC_SCRATCH_BYTES, stream) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
@@ -630,7 +675,7 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
   DeviceInfo* dev = nullptr;
   int st = device_setup(&dev);
   if (st != W4A4_OK) return st;
-  void* scratch = noalloc_scratch();
+  void* scratch = noalloc_scratch(static_cast<cudaStream_t>(stream));
   if (scratch == nullptr) return W4A4_ERR_CUDA;
   return nvfp4_quantize_act(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, scratch,
                             W4A4_NOALLOC_SCRATCH_BYTES, stream);

@@ -88,7 +88,15 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
 
 /* Workspace bytes needed by nvfp4_quantize_act / nvfp4_pack_weight for an
  * [M, K] input with rank r (amax partial maxima, low-rank partial sums and
- * per-row-block counters).  Returns 0 for invalid sizes. */
+ * per-row-block counters).  Returns 0 for invalid sizes.
+ *
+ * Workspace contract (every entry point that takes a workspace): zero the
+ * whole workspace once before its first use (cudaMemset, torch.zeros).  The
+ * counters in it are zero at rest: each call clears the ones it used before
+ * its last kernel ends, so no clearing is needed between calls, whatever
+ * their sizes.  After a call reports a device error (w4a4_device_status),
+ * zero the workspace again.  Calls that overlap on the GPU must not share a
+ * workspace. */
 size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r);
 
 /* Workspace bytes needed by w4a4_linear: the quantisation workspace plus the
@@ -112,7 +120,8 @@ size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  *   t_x    out  fp32 device scalar, the activation's tensor scale
  *   U      out  bf16 [M, 2r] hi/lo low-rank activations (NULL iff r == 0)
  *   workspace   >= nvfp4_quant_workspace_bytes(M, K, r) bytes of device memory,
- *               contents need not be initialised; must not overlap the outputs
+ *               zeroed before its first use (see nvfp4_quant_workspace_bytes);
+ *               must not overlap the outputs
  * Launches one cooperative kernel (tensor amax, grid barrier, quantise and
  * down-projection) when every (128-row block, K slice) tile of X fits on the
  * device at once, otherwise two (tensor amax, then quantise + down-projection).
@@ -131,7 +140,7 @@ int nvfp4_quantize_act(const void* X, int64_t M, int64_t K, int64_t ldx,
  * nvfp4_quantize_act plus
  *   amax  in  fp32 device scalar (4-byte aligned), A >= 0
  * W4A4_ERR_NULL if amax is NULL, W4A4_ERR_ALIGN if misaligned.  Launches one
- * quantise kernel (preceded by a small memset when r > 0).
+ * quantise kernel.
  */
 int nvfp4_quantize_act_with_amax(const void* X, int64_t M, int64_t K, int64_t ldx,
                                  const float* inv_s, const void* L1t, int r, const float* t_w,
@@ -164,6 +173,9 @@ int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_
  *   Wq/Wsf/t_w    in  as written by nvfp4_pack_weight
  *   L2t  in  bf16 [N, r] (NULL iff r == 0);  bias in bf16 [N] or NULL
  *   Y    out bf16 [M, ldy], ldy >= N, ldy % 8 == 0
+ * The kernel is launched with programmatic stream serialisation: its set-up
+ * (barriers, TMEM allocation) overlaps the end of the previous kernel in the
+ * stream, and it touches no memory before that kernel has completed.
  */
 int w4a4_gemm(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U,
               int64_t M, int64_t N, int64_t K,
@@ -225,13 +237,14 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K,
  *   before anything is enqueued (with r = 32 this admits roughly M up to
  *   100k tokens).
  * - The first call on a device looks up the device address of the array
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current), caches it and zeroes
+ *   the array on that call's stream; make that first call before any stream
+ *   capture.
  * - All calls share the one array, which keeps the last call's contents.  The
- *   kernels rewrite every scratch value they read and clear the counters at
- *   the start of each call, so no clearing is needed between calls, but calls
- *   that overlap on the GPU (for example on two streams without ordering
- *   between them) race on the array and give wrong results.
+ *   kernels rewrite every scratch value they read and leave the counters zero
+ *   when they end, so no clearing is needed between calls, but calls that
+ *   overlap on the GPU (for example on two streams without ordering between
+ *   them) race on the array and give wrong results.
  */
 #define W4A4_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
