@@ -20,7 +20,7 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_pack_weight", "w4a4_gemm", "w4a4_linear", "w4a4_device_status",
     "w4a4_status_string", "EPI_NONE", "EPI_GELU_TANH", "SRC_BF16", "SRC_F32",
     "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
-    "new_workspace",
+    "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -48,6 +48,7 @@ _SIG = {
     "w4a4_linear": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _c.c_int, _P, _c.c_int, _P,
                                _P, _c.c_size_t, _P]),
     "w4a4_device_status": (_c.c_int, [_c.POINTER(_c.c_int), _c.c_int]),
+    "nvfp4_sf_to_rowmajor": (_c.c_int, [_P, _I64, _I64, _P, _P]),
     "w4a4_status_string": (_c.c_char_p, [_c.c_int]),
 }
 
@@ -152,6 +153,18 @@ def w4a4_linear(X, M, N, K, Wq, Wsf, t_w, inv_s, L1t, L2t, r, bias, epilogue, Y,
         _ptr(X), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(inv_s), _ptr(L1t), _ptr(L2t), r, _ptr(bias),
         epilogue, _ptr(Y), _ptr(workspace),
         workspace.numel() * workspace.element_size() if workspace is not None else 0, _stream(stream)))
+
+
+def nvfp4_sf_to_rowmajor(sf_atoms, rows, K, sf_rowmajor, stream=None):
+    _check("nvfp4_sf_to_rowmajor", lib().nvfp4_sf_to_rowmajor(
+        _ptr(sf_atoms), rows, K, _ptr(sf_rowmajor), _stream(stream)))
+
+
+def sf_rowmajor(sf_atoms: torch.Tensor, rows: int, K: int, stream=None) -> torch.Tensor:
+    """The scale bytes of an SF-atom buffer as a row-major [rows, K/16] uint8 tensor."""
+    out = torch.empty(rows, K // 16, dtype=torch.uint8, device=sf_atoms.device)
+    nvfp4_sf_to_rowmajor(sf_atoms, rows, K, out, stream)
+    return out
 
 
 def w4a4_device_status(reset: bool = False) -> int:

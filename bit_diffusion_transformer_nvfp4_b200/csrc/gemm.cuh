@@ -45,6 +45,7 @@ struct GemmParams {
   const __nv_bfloat16* bias;
   __nv_bfloat16* Y;
   int has_lr;
+  int r;  // low-rank rank: 0, 16 or 32
   int epi;
   int* status;
   // optional: the next layer's tensor amax max |fl(y * next_inv_s)| over the
@@ -54,6 +55,17 @@ struct GemmParams {
   const float* next_inv_s;
   unsigned* next_amax;
 };
+
+// Shared-memory descriptors of the low-rank pass, K step k (16 columns) of
+// U = [hi | lo] (rows of 2r bf16: 128-byte swizzle at rank 32, 64-byte at
+// rank 16) against L2t (rows of r bf16: 64-byte / 32-byte swizzle), whose
+// columns are used once for the hi and once for the lo half.
+__device__ __forceinline__ uint64_t lowrank_desc_u(uint32_t base, int k, int r) {
+  return r == 32 ? smem_desc(base + 32 * k, 16, 1024, kSwizzle128B) : smem_desc(base + 32 * k, 16, 512, kSwizzle64B);
+}
+__device__ __forceinline__ uint64_t lowrank_desc_l2(uint32_t base, int k, int r) {
+  return r == 32 ? smem_desc(base + 32 * (k & 1), 16, 512, kSwizzle64B) : smem_desc(base, 16, 256, kSwizzle32B);
+}
 
 // Fold eight stored bf16 outputs (columns n .. n+7) into a running amax of
 // |y * s| (s > 0, so |fl(y s)| = fl(|y| s)).
@@ -95,7 +107,7 @@ struct GemmCfg {
   static constexpr int SFA_BYTES = 4 * 512;            // 4 atoms (one per K=64)
   static constexpr int SFB_BYTES = 2 * 4 * 512;        // 2 row blocks x 4 atoms
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int LR_BYTES = BM * 128 + BN * 64;  // U tile + L2t tile
+  static constexpr int LR_BYTES = BM * 128 + BN * 64;  // U tile + L2t tile at rank 32 (rank 16: half)
   static constexpr int NUM_ACC = (2 * BN + 48 <= 512) ? 2 : 1;
   static constexpr int SFA_COL = NUM_ACC * BN;
   static constexpr int SFB_COL = SFA_COL + 16;
@@ -208,7 +220,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* st = smem + s * C::STAGE_BYTES;
           const uint32_t bar = smem_u32(&full[s]);
-          mbar_arrive_expect_tx(bar, C::LR_BYTES);
+          mbar_arrive_expect_tx(bar, C::LR_BYTES * p.r / 32);
           tma_load_2d(smem_u32(st), &tm_u, bar, 0, m0);
           tma_load_2d(smem_u32(st + C::A_BYTES), &tm_l2, bar, 0, n0);
           ++it;
@@ -258,9 +270,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const uint32_t b_base = a_base + C::A_BYTES;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(b_base + 32 * (k & 1), 16, 512, kSwizzle64B);
-            mma_bf16(d, ad, bd, kIdescBf, k > 0 ? 1u : 0u);
+            if (k < p.r / 8) mma_bf16(d, lowrank_desc_u(a_base, k, p.r), lowrank_desc_l2(b_base, k, p.r), kIdescBf, k > 0 ? 1u : 0u);
           }
           tc_commit(smem_u32(&empty[s]));
           ++it;

@@ -45,7 +45,7 @@ struct Gemm2Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BH * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int LR_BYTES = BM * 128 + BH * 64;  // U tile + this CTA's L2t half
+  static constexpr int LR_BYTES = BM * 128 + BH * 64;  // U tile + this CTA's L2t half at rank 32 (rank 16: half)
   // scale ring: one slot per 256-deep K step, this CTA's 128 rows of A
   // scales (4 atoms) and the weight scales of every 128-row block the tile
   // touches (a 192-wide tile may start 64 rows into a block)
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* st = smem + s * C::STAGE_BYTES;
           const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * C::LR_BYTES);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * C::LR_BYTES * p.r / 32);
           tma_load_2d_pair(smem_u32(st), &tm_u, bar, 0, m0);
           tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tm_l2, bar, 0, nb0);
           ++it;
@@ -262,9 +262,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const uint32_t b_base = a_base + C::A_BYTES;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(b_base + 32 * (k & 1), 16, 512, kSwizzle64B);
-            mma_bf16_pair(d, ad, bd, kIdescBf, k > 0 ? 1u : 0u);
+            if (k < p.r / 8)
+              mma_bf16_pair(d, lowrank_desc_u(a_base, k, p.r), lowrank_desc_l2(b_base, k, p.r), kIdescBf, k > 0 ? 1u : 0u);
           }
           tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);
           ++it;

@@ -152,6 +152,7 @@ struct QuantParams {
   int splits;
   int row_blocks;
   int has_lr;
+  int r;                   // low-rank rank (16 or 32) when has_lr
   int* status;
 };
 
@@ -235,14 +236,16 @@ __device__ __forceinline__ float tensor_scale_from(float amax) {
 }
 
 // The last K slice of a row block sums the fp32 partials in slice order,
-// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row (columns in
-// two halves of 16, two slices' loads in flight).
+// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row (row of 2r
+// bf16: hi in columns [0, r), lo in [r, 2r); columns in groups of 16, two
+// slices' loads in flight).
 __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, int64_t rows_pad, int64_t prow,
                                                  int64_t row) {
   __threadfence();
   const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
+  __nv_bfloat16* urow = p.u_out + row * 2 * p.r;
 #pragma unroll 1
-  for (int hh = 0; hh < 2; ++hh) {
+  for (int hh = 0; hh < p.r / 16; ++hh) {
     float acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
@@ -279,11 +282,12 @@ __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, 
         hi[j / 2] = h;
         lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
       }
-      uint4* dst = reinterpret_cast<uint4*>(p.u_out + row * 64 + 16 * hh);
-      dst[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      dst[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-      dst[4] = make_uint4(lo[0], lo[1], lo[2], lo[3]);  // the lo half starts 32 columns on
-      dst[5] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+      uint4* dh = reinterpret_cast<uint4*>(urow + 16 * hh);
+      uint4* dl = reinterpret_cast<uint4*>(urow + p.r + 16 * hh);
+      dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      dh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+      dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
     }
   }
 }
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
           uint8_t* dst = smem + s * Tile::kStageBytes;
           const int kx = (kc0 + i) * kQChunk;
           if constexpr (sizeof(SrcT) == 2) {
-            mbar_arrive_expect_tx(bar, Tile::kBytes + (lr ? Tile::kL1Bytes : 0) + inv_bytes);
+            mbar_arrive_expect_tx(bar, Tile::kBytes + (lr ? 2 * kQChunk * p.r : 0) + inv_bytes);
             tma_load_2d(smem_u32(dst), &tm_x, bar, kx, rb * kQRows);
             if (lr) tma_load_2d(smem_u32(dst + Tile::kL1Off), &tm_l1, bar, kx, 0);
           } else {
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
           for (int k = 0; k < 4; ++k) {
             const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
             const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
-            mma_bf16(d, ad, bd, idesc_bf16(128, 32), (i > 0 || k > 0) ? 1u : 0u);
+            mma_bf16(d, ad, bd, idesc_bf16(128, p.r), (i > 0 || k > 0) ? 1u : 0u);
           }
           tc_commit(smem_u32(&mma_done[s]));
         }
@@ -589,6 +593,19 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
   }
 }
 
+// ------------------------------------------------------------------ layout helper
+// SF atoms -> row-major [rows, K/16]: one thread per (row, 64-wide K group);
+// the group's four scale bytes of a row are one 32-bit word of its atom.
+__global__ void sf_to_rowmajor_kernel(const uint8_t* __restrict__ atoms, int64_t rows, int64_t groups,
+                                      uint8_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * groups) return;
+  const int64_t m = i / groups, g = i % groups;
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(atoms + ((m / kQRows) * groups + g) * 512 + (m % 32) * 16 +
+                                                         ((m / 32) % 4) * 4);
+  *reinterpret_cast<uint32_t*>(out + (m * groups + g) * 4) = w;
+}
+
 // ------------------------------------------------------------------ fused single pass
 // When every (128-row block, K slice) tile of the activation fits in the
 // shared memory of one co-resident wave of CTAs (one CTA per SM, up to
@@ -719,7 +736,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       auto load_l1 = [&](int c) {
         const int s = c % kFusedL1Ring;
         const uint32_t bar = smem_u32(&l1_full[s]);
-        mbar_arrive_expect_tx(bar, 32 * kQChunk * 2);
+        mbar_arrive_expect_tx(bar, p.r * kQChunk * 2);
         tma_load_2d(smem_u32(l1s + s * 32 * kQChunk * 2), &tm_l1, bar, (kc0 + c) * kQChunk, 0);
       };
       for (int c = 0; c < n; ++c) {
@@ -751,7 +768,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         for (int k = 0; k < 4; ++k) {
           const uint64_t ad = smem_desc(a_base + 32 * k, 16, 1024, kSwizzle128B);
           const uint64_t bd = smem_desc(b_base + 32 * k, 16, 1024, kSwizzle128B);
-          mma_bf16(tmem, ad, bd, idesc_bf16(128, 32), (c > 0 || k > 0) ? 1u : 0u);
+          mma_bf16(tmem, ad, bd, idesc_bf16(128, p.r), (c > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit(smem_u32(&l1_empty[s]));
       }
@@ -796,14 +813,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (!*abort_flag) {
           // -------------------------------------------------- this CTA's share of the U rows
           // The slices of a row block split its 128 rows; four threads per
-          // row, eight columns each; the sum runs in slice order.
+          // row, eight columns each (r / 8 of them busy); the sum runs in
+          // slice order.
           const float t = *t_shared;
           const int ut = tid - 32 * kFUWarp0;
           const int cg = ut & 3;
           const int rows_per = (kQRows + p.splits - 1) / p.splits;
           const int r_end = min(kQRows, (split + 1) * rows_per);
           const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
-          for (int rr = split * rows_per + (ut >> 2); rr < r_end; rr += 32) {
+          for (int rr = split * rows_per + (ut >> 2); cg < p.r / 8 && rr < r_end; rr += 32) {
             const int64_t prow2 = static_cast<int64_t>(rb) * kQRows + rr;
             float acc[8];
 #pragma unroll
@@ -841,9 +859,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 hi[j / 2] = hb;
                 lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(hb)), __fsub_rn(a1, bf16_hi(hb)));
               }
-              __nv_bfloat16* urow = p.u_out + prow2 * 64;
+              __nv_bfloat16* urow = p.u_out + prow2 * 2 * p.r;
               *reinterpret_cast<uint4*>(urow + cg * 8) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-              *reinterpret_cast<uint4*>(urow + 32 + cg * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+              *reinterpret_cast<uint4*>(urow + p.r + cg * 8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
           }
         }

@@ -264,7 +264,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
 }
-constexpr uint32_t kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle64B = 4;
+constexpr uint32_t kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle64B = 4, kSwizzle32B = 6;
 
 // Instruction descriptors.  Field positions: [4,6) D format (1 = fp32, for
 // kind::f16), [7,10) A format, [10,13) B format, [15] / [16] A / B major

@@ -224,6 +224,7 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   p.splits = splits;
   p.row_blocks = static_cast<int>(rb);
   p.has_lr = r > 0 ? 1 : 0;
+  p.r = r;
   p.status = dev->status_ptr;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(rb * splits), 1, 1);
@@ -312,6 +313,7 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   p.splits = plan.splits;
   p.row_blocks = static_cast<int>(plan.row_blocks);
   p.has_lr = r > 0 ? 1 : 0;
+  p.r = r;
   p.status = dev->status_ptr;
   // persistent: one CTA per SM walks the (row block, K slice) work items
   const int64_t items = plan.row_blocks * plan.splits;
@@ -337,11 +339,14 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   if (!encode_sf(&tsa, Xsf, M, K, 1)) return W4A4_ERR_CUDA;
   if (!encode_sf(&tsb, Wsf, N, K, 2)) return W4A4_ERR_CUDA;
   if (r > 0) {
-    if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, 64u, static_cast<uint64_t>(M), 128u, 64u, 128u,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    // U = [hi | lo], rows of 2r bf16; L2t rows of r bf16 (swizzle = row width)
+    if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, static_cast<uint64_t>(2 * r), static_cast<uint64_t>(M),
+                   static_cast<uint64_t>(4 * r), static_cast<uint32_t>(2 * r), 128u,
+                   r == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return W4A4_ERR_CUDA;
-    if (!encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2t, 32u, static_cast<uint64_t>(N), 64u, 32u,
-                   static_cast<uint32_t>(C::BN), CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2t, static_cast<uint64_t>(r), static_cast<uint64_t>(N),
+                   static_cast<uint64_t>(2 * r), static_cast<uint32_t>(r), static_cast<uint32_t>(C::BN),
+                   r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
       return W4A4_ERR_CUDA;
   } else {
     tu = ta;
@@ -357,6 +362,7 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.has_lr = r > 0 ? 1 : 0;
+  p.r = r;
   p.epi = epi;
   p.status = dev->status_ptr;
   p.next_inv_s = next_inv_s;
@@ -399,11 +405,14 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
                  static_cast<uint64_t>(ldy) * 2, 32u, 32u, CU_TENSOR_MAP_SWIZZLE_64B))
     return W4A4_ERR_CUDA;
   if (r > 0) {
-    if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, 64u, static_cast<uint64_t>(M), 128u, 64u, 128u,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    // U = [hi | lo], rows of 2r bf16; L2t rows of r bf16 (swizzle = row width)
+    if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, static_cast<uint64_t>(2 * r), static_cast<uint64_t>(M),
+                   static_cast<uint64_t>(4 * r), static_cast<uint32_t>(2 * r), 128u,
+                   r == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return W4A4_ERR_CUDA;
-    if (!encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2t, 32u, static_cast<uint64_t>(N), 64u, 32u,
-                   static_cast<uint32_t>(C::BH), CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L2t, static_cast<uint64_t>(r), static_cast<uint64_t>(N),
+                   static_cast<uint64_t>(2 * r), static_cast<uint32_t>(r), static_cast<uint32_t>(C::BH),
+                   r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B))
       return W4A4_ERR_CUDA;
   } else {
     tu = ta;
@@ -419,6 +428,7 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.has_lr = r > 0 ? 1 : 0;
+  p.r = r;
   p.epi = epi;
   p.status = dev->status_ptr;
   p.next_inv_s = next_inv_s;
@@ -452,7 +462,7 @@ int check_gemm_args(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
                     const void* bias, int epi, const void* Y, int64_t ldy) {
   if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || M > (int64_t(1) << 30) || N > (int64_t(1) << 30))
     return W4A4_ERR_SHAPE;
-  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
   if (epi != W4A4_EPI_NONE && epi != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
   if (ldy < N || ldy % 8 != 0) return W4A4_ERR_SHAPE;
   if (!Xq || !Xsf || !t_x || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
@@ -476,12 +486,12 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
 }
 
 size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r) {
-  if (M < 0 || !valid_k(K) || (r != 0 && r != 32)) return 0;
+  if (M < 0 || !valid_k(K) || (r != 0 && r != 16 && r != 32)) return 0;
   return quant_plan(M, K, r).bytes;
 }
 
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
-  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || (r != 0 && r != 32)) return 0;
+  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || (r != 0 && r != 16 && r != 32)) return 0;
   size_t b = quant_plan(M, K, r).bytes;
   b += round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));  // Xq
   b += round256(nvfp4_sf_bytes(M, K));                                  // Xsf
@@ -494,7 +504,7 @@ static int quantize_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, c
                              int r, const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* workspace,
                              size_t workspace_bytes, void* stream, const float* amax_in) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
-  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
   if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;
   if (r > 0 && (!L1t || !t_w || !U)) return W4A4_ERR_NULL;
   if (!aligned16(X) || !aligned16(Xq) || !aligned16(Xsf) || (inv_s && !aligned16(inv_s)) ||
@@ -592,7 +602,7 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* W
                 const float* t_w, const float* inv_s, const void* L1t, const void* L2t, int r, const void* bias,
                 int epilogue, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
   if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
-  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
   if (epilogue != W4A4_EPI_NONE && epilogue != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
   if (!X || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
   if (r > 0 && (!L1t || !L2t)) return W4A4_ERR_NULL;
@@ -611,6 +621,22 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* W
   int st = nvfp4_quantize_act(X, M, K, K, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, workspace, plan.bytes, stream);
   if (st != W4A4_OK) return st;
   return w4a4_gemm(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, N, stream);
+}
+
+int nvfp4_sf_to_rowmajor(const uint8_t* sf_atoms, int64_t rows, int64_t K, uint8_t* sf_rowmajor, void* stream) {
+  if (rows < 0 || !valid_k(K) || rows > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
+  if (rows == 0) return W4A4_OK;
+  if (!sf_atoms || !sf_rowmajor) return W4A4_ERR_NULL;
+  if (!aligned16(sf_atoms) || !aligned16(sf_rowmajor)) return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  const int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  const int64_t n = rows * (K / kQChunk);
+  const int64_t blocks = ceil_div(n, 256);
+  sf_to_rowmajor_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      sf_atoms, rows, K / kQChunk, sf_rowmajor);
+  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  return W4A4_OK;
 }
 
 int w4a4_device_status(int* status, int reset) {
@@ -667,7 +693,7 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
                                int r, const float* t_w, uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U,
                                void* stream) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
-  if (r != 0 && r != 32) return W4A4_ERR_SHAPE;
+  if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
   const size_t need = nvfp4_quant_workspace_bytes(M, K, r);
   if (need > W4A4_NOALLOC_SCRATCH_BYTES) return W4A4_ERR_SCRATCH_LIMIT;
   if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;

@@ -47,7 +47,9 @@
  *     the legacy default stream).  Scalars (t_x, t_w) stay in device memory.
  *   - Host-detectable problems return an error before anything is enqueued.
  *   - Pointers must be 16-byte aligned; ldx/ldr/ldy are in elements.
- *   - Constraints: K % 256 == 0, K >= 256; N % 8 == 0; r in {0, 32};
+ *   - Constraints: K % 256 == 0, K >= 256; N % 8 == 0; r in {0, 16, 32}
+ *     (rank 16 is the pages' choice for the low-rank branch, "SVDQuant
+ *     Guide ...", "The Solution ..." and "Empirical Efficiency Benchmark");
  *     M >= 0 (M == 0 is a no-op), rows need not be a multiple of 128.
  *   - A device-side pipeline wait that exceeds its bound (about two seconds)
  *     records W4A4_ERR_DEVICE_TIMEOUT in a sticky status word, drains its own
@@ -255,6 +257,17 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
  * (W4A4_OK, W4A4_ERR_DEVICE_TIMEOUT or W4A4_ERR_DEVICE_LAYOUT) and clears it if reset != 0.  This call
  * synchronises the device.  Returns W4A4_OK or W4A4_ERR_CUDA. */
 int w4a4_device_status(int* status, int reset);
+
+/*
+ * nvfp4_sf_to_rowmajor -- a layout helper (for checking and debugging): the
+ * block-scale bytes of an SF-atom buffer (nvfp4_sf_bytes(rows, K) bytes, as
+ * written by nvfp4_quantize_act / nvfp4_pack_weight) rearranged row-major,
+ * sf_rowmajor[m * (K/16) + k/16] = the E4M3 scale of row m, K-block k/16, for
+ * the first ``rows`` rows (the atom layout's pad rows are dropped).  Device
+ * pointers, stream-ordered, one kernel.  W4A4_ERR_SHAPE for invalid sizes,
+ * W4A4_ERR_NULL / W4A4_ERR_ALIGN for bad pointers (16-byte alignment).
+ */
+int nvfp4_sf_to_rowmajor(const uint8_t* sf_atoms, int64_t rows, int64_t K, uint8_t* sf_rowmajor, void* stream);
 
 /* Static description of a status code; never NULL. */
 const char* w4a4_status_string(int status);

@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ["nvfp4_quantize_act", "nvfp4_pack_weight", "w4a4_gemm", "w4a4_linear", "nvfp4_sf_bytes",
               "nvfp4_quant_workspace_bytes", "w4a4_workspace_bytes", "w4a4_device_status",
-              "w4a4_status_string"]:
+              "w4a4_status_string", "nvfp4_sf_to_rowmajor"]:
         assert n in names
 
 
@@ -46,7 +46,8 @@ def test_sizes(so):
     assert so.nvfp4_sf_bytes(10, 100) == 0
     assert so.nvfp4_quant_workspace_bytes(4608, 3072, 32) > 4608 * 32 * 4
     assert so.nvfp4_quant_workspace_bytes(4608, 3000, 32) == 0
-    assert so.nvfp4_quant_workspace_bytes(4608, 3072, 16) == 0
+    assert so.nvfp4_quant_workspace_bytes(4608, 3072, 16) > 0
+    assert so.nvfp4_quant_workspace_bytes(4608, 3072, 24) == 0
     ws = so.w4a4_workspace_bytes(4608, 9216, 3072, 32)
     assert ws >= 4608 * 1536 + 4608 * 192 + 4608 * 128
     assert so.w4a4_workspace_bytes(4608, 9210, 3072, 32) == 0
@@ -66,7 +67,8 @@ def test_host_validation_before_any_launch(so):
     assert q(None, 128, 512, 512, None, None, 0, None, P, P, P, None, P, big, None) == -1     # NULL X
     assert q(P, 128, 500, 512, None, None, 0, None, P, P, P, None, P, big, None) == -2        # K % 256
     assert q(P, 128, 512, 500, None, None, 0, None, P, P, P, None, P, big, None) == -2        # ldx < K
-    assert q(P, 128, 512, 512, None, None, 16, None, P, P, P, None, P, big, None) == -2       # rank
+    assert q(P, 128, 512, 512, None, None, 24, None, P, P, P, None, P, big, None) == -2       # rank
+    assert q(P, 128, 512, 512, None, None, 16, None, P, P, P, None, P, big, None) == -1       # rank 16, no L1t
     assert q(P, 128, 512, 512, None, None, 32, None, P, P, P, None, P, big, None) == -1       # no L1t
     assert q(P + 2, 128, 512, 512, None, None, 0, None, P, P, P, None, P, big, None) == -3    # alignment
     assert q(P, 128, 512, 512, None, None, 0, None, P, P, P, None, P, 16, None) == -5         # workspace
@@ -75,6 +77,10 @@ def test_host_validation_before_any_launch(so):
     assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 7, P, 128, None) == -8     # epilogue
     assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 120, None) == -2     # ldy < N
     assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 32, None, 0, P, 128, None) == -1    # no U/L2t
+    h = w.lib().nvfp4_sf_to_rowmajor
+    assert h(P, 128, 500, P, None) == -2                                                      # K % 256
+    assert h(None, 128, 512, P, None) == -1                                                   # NULL
+    assert h(P, 128, 512, P + 4, None) == -3                                                  # alignment
     pw = w.lib().nvfp4_pack_weight
     assert pw(P, 5, 128, 512, 512, P, P, P, P, big, None) == -8                               # dtype
 

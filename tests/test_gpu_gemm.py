@@ -71,6 +71,8 @@ def run_case(w4, c, rows=None, epilogue=0, use_linear=True, exact_svd=None):
     (257, 768, 576, 0, True),       # no low-rank branch
     (1, 256, 512, 32, True),        # a single token
     (640, 1024, 1024, 32, True),    # several tiles per CTA row
+    (300, 512, 384, 16, True),      # rank 16, CTA pairs
+    (100, 768, 264, 16, True),      # rank 16, single-CTA kernel, ragged N
 ])
 def test_gemm_small(w4, M, K, N, r, bias):
     c = make_linear("t", M, K, N, r=r, act="normal_outliers", n_out=4, out_scale=100.0,

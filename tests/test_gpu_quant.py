@@ -87,14 +87,29 @@ def test_quant_shapes_with_smoothing(w4, M, K):
     check_bytes(x, inv_s, xq, sf, t)
 
 
-def test_quant_lowrank_u(w4):
-    c = make_linear("t", 300, 512, 384, r=32, act="normal_outliers", n_out=6, out_scale=100.0, seed=5)
-    p = prepare(c)
-    qa, xq, sf, t = run_quant(w4, c.x, p["inv_s"], p["L1t"], float(p["t_w"]))
-    check_bytes(c.x, p["inv_s"], xq, sf, t)
+@pytest.mark.parametrize("M,K,r,given", [
+    (300, 512, 32, False),     # single pass
+    (300, 512, 16, False),     # single pass, rank 16
+    (300, 512, 16, True),      # streaming pass with the amax given, rank 16
+    (2048, 12288, 16, False),  # two passes (the tile set is not co-resident), rank 16
+])
+def test_quant_lowrank_u(w4, M, K, r, given):
     import torch
+    c = make_linear("t", M, K, 384, r=r, act="normal_outliers", n_out=6, out_scale=100.0, seed=5 + r)
+    p = prepare(c)
+    if given:
+        a = np.max(np.abs((c.x * p["inv_s"][None, :]).astype(np.float32)))
+        qa = w4.quantize_act(to_dev_bf16(c.x), to_dev_f32(p["inv_s"]), to_dev_bf16(p["L1t"]),
+                             to_dev_f32(np.array([p["t_w"]], np.float32)), amax=to_dev_f32(np.array([a], np.float32)))
+        torch.cuda.synchronize()
+        assert w4.w4a4_device_status() == 0
+        xq, sf, t = qa.Xq.cpu().numpy(), sf_atoms_to_rowmajor(qa.Xsf.cpu().numpy(), M, K), float(qa.t_x.cpu()[0])
+    else:
+        qa, xq, sf, t = run_quant(w4, c.x, p["inv_s"], p["L1t"], float(p["t_w"]))
+    check_bytes(c.x, p["inv_s"], xq, sf, t)
+    assert tuple(qa.U.shape) == (M, 2 * r)
     U = qa.U.float().cpu().numpy()
-    hi, lo = U[:, :32], U[:, 32:]
+    hi, lo = U[:, :r], U[:, r:]
     alpha = np.float64(np.float32(np.float32(t) * np.float32(p["t_w"])))
     ref = olinear.lowrank_down(c.x, p["L1t"]) / alpha
     got = hi.astype(np.float64) + lo.astype(np.float64)
@@ -105,6 +120,22 @@ def test_quant_lowrank_u(w4):
     # hi holds the leading bf16 part: |lo| is at most half a bf16 ulp of hi
     # (plus lo's own rounding)
     assert np.all(np.abs(lo) <= np.abs(hi) * 2.0 ** -8 * (1 + 2.0 ** -7))
+
+
+def test_sf_to_rowmajor_entry(w4):
+    """The C-ABI layout helper equals the test's own numpy rearrangement of
+    the SF atoms, on activation scales (ragged rows) and weight scales."""
+    import torch
+    g = rng(77)
+    x = bf16_round(g.standard_normal((300, 768)).astype(np.float32) * 3.0)
+    qa = w4.quantize_act(to_dev_bf16(x))
+    got = w4.sf_rowmajor(qa.Xsf, 300, 768)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(got.cpu().numpy(), sf_atoms_to_rowmajor(qa.Xsf.cpu().numpy(), 300, 768)[:300])
+    pw = w4.pack_weight(to_dev_f32(g.standard_normal((520, 512)).astype(np.float32)))
+    got = w4.sf_rowmajor(pw.Wsf, 520, 512)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(got.cpu().numpy(), sf_atoms_to_rowmajor(pw.Wsf.cpu().numpy(), 520, 512)[:520])
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
