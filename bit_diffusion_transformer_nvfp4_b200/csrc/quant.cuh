@@ -616,6 +616,7 @@ __global__ void sf_to_rowmajor_kernel(const uint8_t* __restrict__ atoms, int64_t
 // the chunks land (L1t streams through a small ring).
 constexpr int kFusedMaxChunks = 12;
 constexpr int kFusedL1Ring = 7;  // L1t tiles in flight: as many as fit beside the resident X
+constexpr int kFusedSlicesForSpread = 16;
 
 struct FusedQuantSmem {
   static constexpr int kXBytes = kFusedMaxChunks * kQRows * kQChunk * 2;   // 192 KB

@@ -80,12 +80,16 @@ int device_setup(DeviceInfo** out) {
                                   FusedQuantSmem::kBytes) == cudaSuccess;
   using G256 = GemmCfg<256, 4>;
   using G192 = GemmCfg<192, 4>;
+
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G256>, cudaFuncAttributeMaxDynamicSharedMemorySize, G256::SMEM) ==
              cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G192>, cudaFuncAttributeMaxDynamicSharedMemorySize, G192::SMEM) ==
              cudaSuccess;
   using P256 = Gemm2Cfg<256, 5>;
   using P192 = Gemm2Cfg<192, 5>;
+  using P64 = Gemm2Cfg<64, 6>;
+  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P64>, cudaFuncAttributeMaxDynamicSharedMemorySize, P64::SMEM) ==
+             cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P256>, cudaFuncAttributeMaxDynamicSharedMemorySize, P256::SMEM) ==
              cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P192>, cudaFuncAttributeMaxDynamicSharedMemorySize, P192::SMEM) ==
@@ -133,7 +137,11 @@ constexpr int kPlanSms = 148;
 // per (row block, slice), at most kFusedMaxChunks chunks each).
 int fused_splits(int64_t row_blocks, int chunks, int64_t sms) {
   int64_t want = ceil_div(chunks, kFusedMaxChunks);
-  const int64_t more = row_blocks > 0 ? sms / row_blocks : 1;
+  // more slices spread the load over more SMs, but every slice adds a
+  // partial U that each row's sum waits for: at most kFusedSlicesForSpread
+  // slices beyond what the shared-memory budget needs
+  int64_t more = row_blocks > 0 ? sms / row_blocks : 1;
+  if (more > kFusedSlicesForSpread) more = kFusedSlicesForSpread;
   if (more > want) want = more;
   if (want > chunks) want = chunks;
   if (want < 1) want = 1;
@@ -568,11 +576,17 @@ static int gemm_dispatch(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x
   if (st != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // CTA pairs (256 x 256 tiles) once there are at least two row blocks;
-  // single-CTA 128 x 192 / 128 x 256 tiles for a single row block.
+  // CTA pairs (256 x 256 tiles) once there are at least two row blocks.
+  // A single row block: CTA pairs with 256 x 64 tiles (the second CTA's rows
+  // are past M: TMA fills them with zeros and the store drops them) while
+  // that gives at most two tiles per pair, so a small layer streams its
+  // weight through many SMs; else single-CTA 128 x 192 / 128 x 256 tiles.
   if (M > 128)
     return launch_gemm_pair<Gemm2Cfg<256, 5>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
                                               next_inv_s, next_amax, s, dev);
+  if (ceil_div(N, 64) <= static_cast<int64_t>(dev->num_sms))
+    return launch_gemm_pair<Gemm2Cfg<64, 6>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
+                                             next_inv_s, next_amax, s, dev);
   if (N % 192 == 0)
     return launch_gemm_cfg<GemmCfg<192, 4>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
                                             next_inv_s, next_amax, s, dev);

@@ -65,7 +65,7 @@ def run_case(w4, c, rows=None, epilogue=0, use_linear=True, exact_svd=None):
 
 
 @pytest.mark.parametrize("M,K,N,r,bias", [
-    (128, 256, 192, 32, True),      # one tile, 192-wide (double-buffered accumulator)
+    (128, 256, 192, 32, True),      # one row block: three 128 x 64 tiles (double-buffered accumulator)
     (300, 512, 384, 32, True),      # ragged M, two N tiles
     (300, 512, 264, 32, False),     # 256-wide tiles, ragged N (264 = 256 + 8)
     (257, 768, 576, 0, True),       # no low-rank branch
@@ -73,6 +73,8 @@ def run_case(w4, c, rows=None, epilogue=0, use_linear=True, exact_svd=None):
     (640, 1024, 1024, 32, True),    # several tiles per CTA row
     (300, 512, 384, 16, True),      # rank 16, CTA pairs
     (100, 768, 264, 16, True),      # rank 16, single-CTA kernel, ragged N
+    (64, 256, 19200, 32, True),     # single row block, wide: 128 x 192 tiles
+    (64, 256, 19456, 0, False),     # single row block, wide: 128 x 256 tiles
 ])
 def test_gemm_small(w4, M, K, N, r, bias):
     c = make_linear("t", M, K, N, r=r, act="normal_outliers", n_out=4, out_scale=100.0,

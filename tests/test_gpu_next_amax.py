@@ -62,7 +62,8 @@ def test_quantize_with_given_amax(w4, M, K, r):
         assert olinear.rel_frobenius(U[:, :32] + U[:, 32:], ref) < 1e-5
 
 
-@pytest.mark.parametrize("M,K,N,gelu", [(640, 3072, 12288, True), (100, 3072, 3072, False), (300, 512, 264, True)])
+@pytest.mark.parametrize("M,K,N,gelu", [(640, 3072, 12288, True), (100, 3072, 3072, False), (300, 512, 264, True),
+                                         (64, 256, 19200, True)])
 def test_gemm_next_amax(w4, M, K, N, gelu):
     import torch
     c = make_linear("up", M, K, N, r=32, act="student_t", bias_std=0.01, seed=M + N)
