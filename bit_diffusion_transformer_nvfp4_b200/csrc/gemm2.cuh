@@ -25,9 +25,12 @@
 //   * the epilogue stages bf16 results in 64-byte-swizzled shared memory and
 //     writes them with TMA stores (full 64-byte rows, clipped at the edges).
 //
-// One persistent CTA pair per two SMs; 448 threads per CTA: warp 0 TMA
-// producer, warp 1 TMEM owner (+ MMA issuer in the even CTA), warps 2-9
-// epilogue, warps 10-13 scale warps.
+// One persistent CTA pair per two SMs; 512 threads per CTA: warp 0 TMA
+// producer, warp 1 TMEM owner (+ MMA issuer in the even CTA), warps 2-3
+// spare, warps 4-7 scale warps, warps 8-15 epilogue.  The launch gives every
+// thread 128 registers; setmaxnreg then shrinks the first two warpgroups and
+// grows the two epilogue warpgroups, whose 128 accumulator columns per thread
+// would otherwise spill.
 #pragma once
 
 #include "gemm.cuh"
@@ -63,8 +66,12 @@ struct Gemm2Cfg {
   static constexpr int NB_TSF = NB_TSF_FIT < 6 ? NB_TSF_FIT : 6;
   static constexpr int TMEM_COLS = 512;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int SF_WARP0 = 2 + EPI_WARPS;       // warps 10-13
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * 4;
+  static constexpr int SF_WARP0 = 4;                   // warps 4-7: scale warps
+  static constexpr int EPI_WARP0 = 8;                  // warps 8-15: epilogue
+  static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+  // registers per thread after setmaxnreg: producer / MMA warpgroup, scale
+  // warpgroup, the two epilogue warpgroups (launch: 65536 / THREADS = 128)
+  static constexpr int REGS_CTRL = 64, REGS_SF = 64, REGS_EPI = 176;
   static constexpr int HALF = BN / 2;                  // columns per epilogue warp
   static constexpr int EPI_BUF = 32 * 64;              // 32 rows x 32 bf16, one staging buffer
   static constexpr int EPI_NBUF = EPI_NBUF_;           // staging buffers per epilogue warp
@@ -83,6 +90,9 @@ struct Gemm2Cfg {
   static_assert(STAGE_BYTES % 1024 == 0 && SF_STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 64 == 0 && HALF % 32 == 0, "tile shape");
+  static_assert(THREADS == 512, "four warpgroups");
+  static_assert(128 * (REGS_CTRL + REGS_SF + 2 * REGS_EPI) <= 65536 - 4096,
+                "register budgets fit the launch allocation with room to spare");
 };
 
 template <class C>
@@ -173,6 +183,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // K steps (with scales) this pair runs: every tile pair, pair+pairs, ...
   const uint32_t total_ks = pair < total ? static_cast<uint32_t>((total - 1 - pair) / pairs + 1) * nkb : 0u;
 
+  // Registers: each role sets its warpgroup's budget first thing (the
+  // control and scale warpgroups give theirs back, the epilogue warpgroups
+  // take them), inside its own branch so that the compiler allocates each
+  // role's code to its budget.
+  if (warp < C::SF_WARP0) regs_release_to<C::REGS_CTRL>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
@@ -300,8 +315,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_wait_drain(smem_u32(drain), 0);
     }
   } else if (warp < C::SF_WARP0) {
+    // spare warps
+  } else if (warp >= C::EPI_WARP0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int ew = warp - 2;
+    regs_grow_to<C::REGS_EPI>();
+    const int ew = warp - C::EPI_WARP0;
     const int q = warp & 3;               // TMEM lane quarter (rows 32q..32q+31 of this CTA)
     const int h = ew >> 2;                // column half
     const float alpha = __fmul_rn(__ldg(p.t_x), __ldg(p.t_w));
@@ -408,6 +426,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ scale warps (both CTAs)
+    regs_release_to<C::REGS_SF>();
     // Lane l holds, per 512-byte atom, the 16 bytes of rows l, l+32, l+64,
     // l+96 (one 32-bit TMEM column per row); every lane quarter gets the same
     // words, so each row's scales sit in its own lane at column 4j + row/32.

@@ -99,6 +99,19 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// --------------------------------------------------------------- register budgets per warpgroup
+// setmaxnreg: every warp of a warpgroup executes the same one; an increase
+// waits until decreases elsewhere in the CTA have freed the registers, so
+// the budgets must add up to no more than the launch's allocation.
+template <int N>
+__device__ __forceinline__ void regs_release_to() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_grow_to() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // --------------------------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialisation may start while
 // the previous kernel in the stream is still running; it must wait here
