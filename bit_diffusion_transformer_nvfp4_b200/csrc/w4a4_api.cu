@@ -473,6 +473,7 @@ int check_gemm_args(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
   if (epi != W4A4_EPI_NONE && epi != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
   if (ldy < N || ldy % 8 != 0) return W4A4_ERR_SHAPE;
+  if (M == 0) return W4A4_OK;  // empty problem
   if (!Xq || !Xsf || !t_x || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
   if (r > 0 && (!U || !L2t)) return W4A4_ERR_NULL;
   if (!aligned16(Xq) || !aligned16(Xsf) || !aligned16(Wq) || !aligned16(Wsf) || !aligned16(Y) ||
@@ -513,6 +514,7 @@ static int quantize_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, c
                              size_t workspace_bytes, void* stream, const float* amax_in) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
+  if (M == 0) return W4A4_OK;  // empty problem: nothing to check further, nothing enqueued
   if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;
   if (r > 0 && (!L1t || !t_w || !U)) return W4A4_ERR_NULL;
   if (!aligned16(X) || !aligned16(Xq) || !aligned16(Xsf) || (inv_s && !aligned16(inv_s)) ||
@@ -522,7 +524,6 @@ static int quantize_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, c
   DeviceInfo* dev = nullptr;
   int st = device_setup(&dev);
   if (st != W4A4_OK) return st;
-  if (M == 0) return W4A4_OK;
   return launch_quant<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(X), M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf,
                                      t_x, U, workspace, static_cast<cudaStream_t>(stream), dev, amax_in);
 }
@@ -538,7 +539,7 @@ int nvfp4_quantize_act_with_amax(const void* X, int64_t M, int64_t K, int64_t ld
                                  const void* L1t, int r, const float* t_w, const float* amax, uint8_t* Xq,
                                  uint8_t* Xsf, float* t_x, void* U, void* workspace, size_t workspace_bytes,
                                  void* stream) {
-  if (!amax) return W4A4_ERR_NULL;
+  if (M != 0 && !amax) return W4A4_ERR_NULL;
   if (reinterpret_cast<uintptr_t>(amax) % 4 != 0) return W4A4_ERR_ALIGN;
   return quantize_act_impl(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, workspace, workspace_bytes, stream,
                            amax);
@@ -549,6 +550,7 @@ int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_
   if (src_dtype != W4A4_SRC_BF16 && src_dtype != W4A4_SRC_F32) return W4A4_ERR_ARG;
   const int64_t vec = src_dtype == W4A4_SRC_BF16 ? 8 : 4;
   if (N < 0 || !valid_k(K) || ldr < K || ldr % vec != 0 || N > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
+  if (N == 0) return W4A4_OK;  // empty problem
   if (!R || !Wq || !Wsf || !t_w) return W4A4_ERR_NULL;
   if (!aligned16(R) || !aligned16(Wq) || !aligned16(Wsf) || (workspace && !aligned16(workspace)))
     return W4A4_ERR_ALIGN;
@@ -556,7 +558,6 @@ int nvfp4_pack_weight(const void* R, int src_dtype, int64_t N, int64_t K, int64_
   DeviceInfo* dev = nullptr;
   int st = device_setup(&dev);
   if (st != W4A4_OK) return st;
-  if (N == 0) return W4A4_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (src_dtype == W4A4_SRC_BF16)
     return launch_quant<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(R), N, K, ldr, nullptr, nullptr, 0, nullptr,
@@ -570,11 +571,10 @@ static int gemm_dispatch(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x
                          const void* bias, int epilogue, void* Y, int64_t ldy, const float* next_inv_s,
                          unsigned* next_amax, void* stream) {
   int st = check_gemm_args(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy);
-  if (st != W4A4_OK) return st;
+  if (st != W4A4_OK || M == 0) return st;
   DeviceInfo* dev = nullptr;
   st = device_setup(&dev);
   if (st != W4A4_OK) return st;
-  if (M == 0) return W4A4_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // CTA pairs (256 x 256 tiles) once there are at least two row blocks.
   // A single row block: CTA pairs with 256 x 64 tiles (the second CTA's rows
@@ -605,7 +605,7 @@ int w4a4_gemm_next_amax(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x,
                         int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
                         const void* bias, int epilogue, void* Y, int64_t ldy, const float* next_inv_s,
                         float* next_amax, void* stream) {
-  if (!next_amax) return W4A4_ERR_NULL;
+  if (M != 0 && !next_amax) return W4A4_ERR_NULL;
   if ((next_inv_s && !aligned16(next_inv_s)) || reinterpret_cast<uintptr_t>(next_amax) % 4 != 0)
     return W4A4_ERR_ALIGN;
   return gemm_dispatch(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, next_inv_s,
@@ -618,6 +618,7 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* W
   if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
   if (epilogue != W4A4_EPI_NONE && epilogue != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
+  if (M == 0) return W4A4_OK;  // empty problem
   if (!X || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
   if (r > 0 && (!L1t || !L2t)) return W4A4_ERR_NULL;
   if (!workspace || workspace_bytes < w4a4_workspace_bytes(M, N, K, r)) return W4A4_ERR_WORKSPACE;
@@ -708,6 +709,7 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
                                void* stream) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
+  if (M == 0) return W4A4_OK;  // empty problem
   const size_t need = nvfp4_quant_workspace_bytes(M, K, r);
   if (need > W4A4_NOALLOC_SCRATCH_BYTES) return W4A4_ERR_SCRATCH_LIMIT;
   if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;

@@ -50,7 +50,10 @@
  *   - Constraints: K % 256 == 0, K >= 256; N % 8 == 0; r in {0, 16, 32}
  *     (rank 16 is the pages' choice for the low-rank branch, "SVDQuant
  *     Guide ...", "The Solution ..." and "Empirical Efficiency Benchmark");
- *     M >= 0 (M == 0 is a no-op), rows need not be a multiple of 128.
+ *     M >= 0, rows need not be a multiple of 128.  An empty problem (M == 0;
+ *     N == 0 for nvfp4_pack_weight; rows == 0 for nvfp4_sf_to_rowmajor) with
+ *     valid sizes returns W4A4_OK at once: pointers may then be NULL,
+ *     nothing is checked further and nothing is enqueued.
  *   - A device-side pipeline wait that exceeds its bound (about two seconds)
  *     records W4A4_ERR_DEVICE_TIMEOUT in a sticky status word, drains its own
  *     copies and returns; read it with w4a4_device_status() after a sync.

@@ -85,6 +85,29 @@ def test_host_validation_before_any_launch(so):
     assert pw(P, 5, 128, 512, 512, P, P, P, P, big, None) == -8                               # dtype
 
 
+def test_empty_problems_are_noops(so):
+    """M == 0 (N == 0 for packing) with valid sizes: W4A4_OK at once, with
+    NULL buffers, no device needed; invalid sizes still fail."""
+    assert so.nvfp4_quantize_act(None, 0, 512, 512, None, None, 32, None, None, None, None, None, None, 0,
+                                 None) == 0
+    assert so.nvfp4_quantize_act_with_amax(None, 0, 512, 512, None, None, 0, None, None, None, None, None, None,
+                                           None, 0, None) == 0
+    assert so.nvfp4_quantize_act_noalloc(None, 0, 512, 512, None, None, 16, None, None, None, None, None,
+                                         None) == 0
+    assert so.w4a4_gemm(None, None, None, None, 0, 128, 512, None, None, None, None, 32, None, 0, None, 128,
+                        None) == 0
+    assert so.w4a4_gemm_next_amax(None, None, None, None, 0, 128, 512, None, None, None, None, 0, None, 1,
+                                  None, 128, None, None, None) == 0
+    assert so.w4a4_linear(None, 0, 128, 512, None, None, None, None, None, None, 16, None, 0, None, None, 0,
+                          None) == 0
+    assert so.nvfp4_pack_weight(None, 1, 0, 512, 512, None, None, None, None, 0, None) == 0
+    assert so.nvfp4_sf_to_rowmajor(None, 0, 512, None, None) == 0
+    assert so.nvfp4_quantize_act(None, 0, 500, 512, None, None, 0, None, None, None, None, None, None, 0,
+                                 None) == -2
+    assert so.w4a4_gemm(None, None, None, None, 0, 100, 512, None, None, None, None, 0, None, 0, None, 100,
+                        None) == -2
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU path")
 def test_no_gpu_reports_arch_error(so):
     P = 1 << 20

@@ -134,3 +134,19 @@ def test_gemm_config2_full_sampled_rows(w4):
     rows[-1] = c.M - 1
     y, y_ref = run_case(w4, c, rows=rows)
     check_y(y, y_ref)
+
+
+def test_empty_batch(w4):
+    """An empty batch (M = 0) through the tensor-level API: no-ops with
+    empty outputs and a clean device status."""
+    import torch
+    c = make_linear("t", 1, 512, 256, r=32, act="normal_outliers", seed=4)
+    p = prepare(c)
+    w = device_weight(w4, p, c.bias, 32)
+    X = torch.empty(0, 512, dtype=torch.bfloat16, device="cuda")
+    qa = w4.quantize_act(X, w.inv_s, w.L1t, w.t_w)
+    Y = w4.gemm(qa, w)
+    Z = w4.linear(X, w)
+    torch.cuda.synchronize()
+    assert tuple(Y.shape) == (0, 256) and tuple(Z.shape) == (0, 256)
+    assert w4.w4a4_device_status() == 0
