@@ -247,26 +247,54 @@ def run_ours(args):
     gemm_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(0, args.steps, MID_EVERY)]
     quant_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(0, args.steps, MID_EVERY)]
 
-    # end to end through the public API with host buffers: pinned X in,
-    # linear on the device, pinned Y out, every step
+    # End to end through the public API with host buffers: every step copies
+    # its X in from pinned host memory, runs w4a4_linear and copies its Y out
+    # to pinned host memory.  Steps are pipelined over three streams (copy in,
+    # compute, copy out) and two device buffer sets, as a serving loop would
+    # run them: one step's copies overlap its neighbours' work, and events keep
+    # the order within a step and the reuse of each buffer set.
     import torch as _t
     xh = _t.from_numpy(x_host).view(_t.bfloat16).pin_memory()
-    yh = _t.empty(M, N, dtype=_t.bfloat16).pin_memory()
+    yh = [_t.empty(M, N, dtype=_t.bfloat16).pin_memory() for _ in range(2)]
     e2e_steps = max(3, min(args.steps, 50))
-    X0, w0, qa0, ws0, Y0 = sets[0]
+    w0 = sets[0][1]
+    bufs = [(sets[j][0], sets[j][4]) for j in range(2)]
     lin_ws = w4.new_workspace(w4.w4a4_workspace_bytes(M, N, K, r), dev)
-    for i in range(2):
-        X0.copy_(xh, non_blocking=True)
-        w4.w4a4_linear(X0, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y0, lin_ws, stream)
-        yh.copy_(Y0, non_blocking=True)
+    s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(n, e_start=None, e_end=None):
+        done_c, done_out = [], []
+        if e_start is not None:
+            e_start.record(s_in)
+        for i in range(n):
+            X, Y = bufs[i % 2]
+            if i >= 2:
+                s_in.wait_event(done_c[i - 2])        # step i-2 no longer reads this X
+            with torch.cuda.stream(s_in):
+                X.copy_(xh, non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+            s_c.wait_event(ev_in)
+            if i >= 2:
+                s_c.wait_event(done_out[i - 2])       # step i-2's Y has been copied out
+            w4.w4a4_linear(X, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y,
+                           lin_ws, s_c)
+            ev_c = torch.cuda.Event()
+            ev_c.record(s_c)
+            s_out.wait_event(ev_c)
+            with torch.cuda.stream(s_out):
+                yh[i % 2].copy_(Y, non_blocking=True)
+            ev_out = torch.cuda.Event()
+            ev_out.record(s_out)
+            done_c.append(ev_c)
+            done_out.append(ev_out)
+        if e_end is not None:
+            e_end.record(s_out)
+
+    e2e_run(4)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        X0.copy_(xh, non_blocking=True)
-        w4.w4a4_linear(X0, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y0, lin_ws, stream)
-        yh.copy_(Y0, non_blocking=True)
-    e1.record(stream)
+    e2e_run(e2e_steps, e0, e1)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     clock_rows = sampler.stop()
@@ -305,7 +333,8 @@ def run_ours(args):
                        "sampled_steps": len(gemm_ms)},
         "e2e": {"value": round(whole_job_tflops(world, fl, 1, e2e_ms), 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2),
-                "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear"},
+                "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear",
+                "pipelining": "copy-in, compute and copy-out on three streams, two buffer sets"},
         # per step: the single-pass quantiser and the pair GEMM
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,

@@ -665,7 +665,7 @@ __device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target,
 
 __global__ void __launch_bounds__(kFThreads, 1)
     quant_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
-                       const QuantParams p, unsigned* grid_sync) {
+                       const __grid_constant__ CUtensorMap tm_q, const QuantParams p, unsigned* grid_sync) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
@@ -921,9 +921,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
     if (tid < 256) rq_tab[tid] = __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(tid)).y, t));
     named_bar_sync(1, 32 * kFComputeWarps);
     const float rt = __frcp_rn(t);
-    const int64_t row = static_cast<int64_t>(rb) * kQRows + r;
-    const bool row_ok = row < p.M;
-    const int64_t kbytes = p.K / 2;
+    // Codes leave through TMA stores of the warp's 32 rows x 32 bytes, staged
+    // in the first kilobyte of the warp's own rows of the chunk it has just
+    // read.  The U MMAs read those tiles too: they are all complete once the
+    // drain barrier has fired (long before this point).
+    if (lr && !mbar_wait(smem_u32(drain), 0, abort_flag, p.status)) return;
+    if (lane == 0) tma_prefetch_desc(&tm_q);
 #pragma unroll
     for (int i = 0; i < kFChunksPerThread; ++i) {
       const int c = grp + kFGroups * i;
@@ -957,15 +960,30 @@ __global__ void __launch_bounds__(kFThreads, 1)
             }
           }
         }
-        if (row_ok) {
-          uint4* dq = reinterpret_cast<uint4*>(p.q + row * kbytes + static_cast<int64_t>(kc) * 32);
-          dq[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          dq[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        // every lane has read its rows of the chunk: stage this warp's codes
+        // (row ``lane`` of 32, 32 bytes; lanes with bit 2 set store their
+        // halves in the other order, no bank conflicts) and store them; the
+        // TMA store drops rows >= M
+        __syncwarp();
+        uint8_t* cb = xs + c * kQRows * kQChunk * 2 + (warp & 3) * 32 * kQChunk * 2;
+        const int first = (lane >> 2) & 1;
+        *reinterpret_cast<uint4*>(cb + lane * 32 + 16 * first) =
+            first ? make_uint4(cw[4], cw[5], cw[6], cw[7]) : make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4*>(cb + lane * 32 + 16 * (first ^ 1)) =
+            first ? make_uint4(cw[0], cw[1], cw[2], cw[3]) : make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_q, smem_u32(cb), kc * 32, rb * kQRows + (warp & 3) * 32);
+          bulk_commit_group();
         }
         const int64_t atom = static_cast<int64_t>(rb) * chunks + kc;
         *reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (r & 31) * 16 + (r >> 5) * 4) = e4;
       }
     }
+    // the code stores have landed before the CTA ends
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
   if (warp == kFProducerWarp && lane == 0) {
     // no copy may still be landing when the CTA exits

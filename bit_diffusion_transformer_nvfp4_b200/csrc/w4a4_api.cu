@@ -215,6 +215,11 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   } else {
     tm_l1 = tm_x;
   }
+  // codes, written by TMA: 32 rows x 32 bytes (one 64-wide chunk) per box
+  CUtensorMap tm_q;
+  if (!encode_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(K / 2), 32u, 32u, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return W4A4_ERR_CUDA;
   QuantParams p;
   p.M = M;
   p.K = K;
@@ -244,7 +249,7 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, p, grid_sync) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, grid_sync) != cudaSuccess) {
     cudaGetLastError();
     return -1;  // not co-resident on this device: fall back
   }
