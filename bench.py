@@ -229,23 +229,30 @@ def run_ours(args):
     for i in range(args.warmup):
         step(i)
     barrier()
-    # Every step is bracketed by events; every MID_EVERY-th step also records
-    # one between the quantiser and the GEMM (for the per-kernel durations).
-    # An event there makes that GEMM wait for the quantiser to finish instead
-    # of starting its set-up early (programmatic launch), so the other steps
-    # go without it.
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # One event pair brackets the timed steps.  Every MID_EVERY-th step also
+    # records events before the quantiser, between the kernels and after the
+    # GEMM (the per-kernel durations).  An event between two kernels makes
+    # the second wait for the first to finish instead of starting its set-up
+    # early (programmatic launch), so the other steps go without them.
+    ev_first, ev_last = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampled = list(range(0, args.steps, MID_EVERY))
+    evs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for i in sampled}
     t_wall0 = time.time()
+    ev_first.record(stream)
     for i in range(args.steps):
-        evs[i][0].record(stream)
-        step(i, evs[i][1] if i % MID_EVERY == 0 else None)
-        evs[i][2].record(stream)
+        if i in evs:
+            evs[i][0].record(stream)
+            step(i, evs[i][1])
+            evs[i][2].record(stream)
+        else:
+            step(i)
+    ev_last.record(stream)
     barrier()
     t_wall1 = time.time()
-    total_ms = evs[0][0].elapsed_time(evs[-1][2])
-    gemm_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(0, args.steps, MID_EVERY)]
-    quant_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(0, args.steps, MID_EVERY)]
+    total_ms = ev_first.elapsed_time(ev_last)
+    gemm_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in sampled]
+    quant_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in sampled]
 
     # End to end through the public API with host buffers: every step copies
     # its X in from pinned host memory, runs w4a4_linear and copies its Y out

@@ -102,6 +102,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                  const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_l2,
                  const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   constexpr int BN = C::BN, STAGES = C::STAGES;
+  // the next kernel in the stream (a programmatic dependent) may be scheduled
+  // on SMs this grid leaves; it waits for this grid's completion itself
+  grid_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = C::ALIGN_BASE
                       ? reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023))

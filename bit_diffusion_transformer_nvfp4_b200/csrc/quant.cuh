@@ -362,6 +362,9 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
     tmem_alloc(smem_u32(tmem_slot), 32 * kQAcc);  // 32-column U accumulators
     tmem_relinquish();
   }
+  // set-up above may overlap the previous kernel (programmatic launch);
+  // nothing below may touch memory before it has completed
+  grid_dependency_wait();
   // tensor scale from the pass-1 partial maxima (the same value in every CTA)
   float m = 0.0f;
   for (int i = tid; i < p.n_partials; i += kQThreads) m = fmaxf(m, p.partials[i]);
@@ -721,6 +724,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = lr ? *tmem_slot : 0u;
+  // set-up above may overlap the previous kernel (programmatic launch);
+  // nothing below may touch memory before it has completed
+  grid_dependency_wait();
 
   float bmax[4 * kFChunksPerThread];  // compute threads: block maxima of their row
   const int r = tid & (kQRows - 1);

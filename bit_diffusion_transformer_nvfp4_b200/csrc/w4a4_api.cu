@@ -244,16 +244,19 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   cfg.blockDim = dim3(kFThreads, 1, 1);
   cfg.dynamicSmemBytes = FusedQuantSmem::kBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, grid_sync) != cudaSuccess) {
-    cudaGetLastError();
-    return -1;  // not co-resident on this device: fall back
-  }
-  return W4A4_OK;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, grid_sync) == cudaSuccess) return W4A4_OK;
+  cudaGetLastError();
+  cfg.numAttrs = 1;  // without the programmatic attribute
+  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, grid_sync) == cudaSuccess) return W4A4_OK;
+  cudaGetLastError();
+  return -1;  // not co-resident on this device: fall back
 }
 
 template <typename SrcT>
@@ -331,9 +334,20 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   // persistent: one CTA per SM walks the (row block, K slice) work items
   const int64_t items = plan.row_blocks * plan.splits;
   const int64_t grid2 = items < dev->num_sms ? items : dev->num_sms;
-  quant_kernel<SrcT><<<static_cast<unsigned>(grid2), kQThreads, QuantTile<SrcT>::kSmem, stream>>>(tm_x, tm_l1, tm_q,
-                                                                                                   p);
-  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid2), 1, 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = QuantTile<SrcT>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, quant_kernel<SrcT>, tm_x, tm_l1, tm_q, p) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
   return W4A4_OK;
 }
 
