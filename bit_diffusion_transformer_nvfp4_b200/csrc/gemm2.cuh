@@ -25,9 +25,9 @@
 //   * the epilogue stages bf16 results in 64-byte-swizzled shared memory and
 //     writes them with TMA stores (full 64-byte rows, clipped at the edges).
 //
-// One persistent CTA pair per two SMs; 512 threads per CTA: warp 0 TMA
-// producer, warp 1 TMEM owner (+ MMA issuer in the even CTA), warps 2-3
-// spare, warps 4-7 scale warps, warps 8-15 epilogue.  The launch gives every
+// One persistent CTA pair per two SMs; 512 threads per CTA: warp 0 A/B TMA
+// producer, warp 1 TMEM owner (+ MMA issuer in the even CTA), warp 2 scale
+// TMA producer, warp 3 spare, warps 4-7 scale warps, warps 8-15 epilogue.  The launch gives every
 // thread 128 registers; setmaxnreg then shrinks the first two warpgroups and
 // grows the two epilogue warpgroups, whose 128 accumulator columns per thread
 // would otherwise spill.
@@ -191,30 +191,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // take them), inside its own branch so that the compiler allocates each
   // role's code to its budget.
   if (warp < C::SF_WARP0) regs_release_to<C::REGS_CTRL>();
+  // scale atoms of K step k (counted over this pair's tiles) into slot k % SF_STAGES
+  auto issue_sf = [&](uint32_t k) -> bool {
+    const int tile = pair + static_cast<int>(k / nkb) * pairs;
+    const int kb = static_cast<int>(k % nkb);
+    const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+    const int n0 = (tile / m_tiles) * BN;
+    const uint32_t slot = k % C::SF_STAGES;
+    if (k >= static_cast<uint32_t>(C::SF_STAGES) &&
+        !mbar_wait(smem_u32(&sf_empty[slot]), ((k / C::SF_STAGES) - 1) & 1, abort_flag, p.status))
+      return false;
+    uint8_t* dst = sf_smem + slot * C::SF_STAGE_BYTES;
+    const uint32_t bar = smem_u32(&sf_full[slot]);
+    mbar_arrive_expect_tx(bar, C::SF_STAGE_BYTES);
+    tma_load_3d(smem_u32(dst), &tm_sfa, bar, 0, kb * 4, m0 / 128);
+    tma_load_3d(smem_u32(dst + C::SFA_BYTES), &tm_sfb, bar, 0, kb * 4, n0 / 128);
+    return true;
+  };
+
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
+    // ------------------------------------------------------------ A/B producer (both CTAs)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      // scale atoms of K step k (counted over this pair's tiles) into slot k % SF_STAGES
-      auto issue_sf = [&](uint32_t k) -> bool {
-        const int tile = pair + static_cast<int>(k / nkb) * pairs;
-        const int kb = static_cast<int>(k % nkb);
-        const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
-        const int n0 = (tile / m_tiles) * BN;
-        const uint32_t slot = k % C::SF_STAGES;
-        if (k >= static_cast<uint32_t>(C::SF_STAGES) &&
-            !mbar_wait(smem_u32(&sf_empty[slot]), ((k / C::SF_STAGES) - 1) & 1, abort_flag, p.status))
-          return false;
-        uint8_t* dst = sf_smem + slot * C::SF_STAGE_BYTES;
-        const uint32_t bar = smem_u32(&sf_full[slot]);
-        mbar_arrive_expect_tx(bar, C::SF_STAGE_BYTES);
-        tma_load_3d(smem_u32(dst), &tm_sfa, bar, 0, kb * 4, m0 / 128);
-        tma_load_3d(smem_u32(dst + C::SFA_BYTES), &tm_sfb, bar, 0, kb * 4, n0 / 128);
-        return true;
-      };
-      uint32_t ksf = 0;
-      while (ksf < total_ks && ksf < static_cast<uint32_t>(C::SF_STAGES)) ok = ok && issue_sf(ksf++);
       for (int tile = pair; tile < total && ok; tile += pairs) {
         const int m0 = (tile % m_tiles) * 2 * C::BM + static_cast<int>(rank) * C::BM;
         const int n0 = (tile / m_tiles) * BN;
@@ -240,13 +239,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tma_load_2d_pair(smem_u32(st), &tm_a, bar, kb * 128, m0);
           tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tm_b, bar, kb * 128, nb0);
           ++it;
-          if (ksf < total_ks && !issue_sf(ksf++)) { ok = false; break; }
         }
       }
-      // no scale copy may still be landing when shared memory goes away
-      const uint32_t sf_first = ksf > static_cast<uint32_t>(C::SF_STAGES) ? ksf - C::SF_STAGES : 0u;
-      for (uint32_t k = sf_first; k < ksf; ++k)
-        mbar_wait_drain(smem_u32(&sf_full[k % C::SF_STAGES]), (k / C::SF_STAGES) & 1);
       // The even CTA's ring barriers count both CTAs' bytes: there, wait
       // (bounded) for the newest fills to land before shared memory goes away.
       if (leader) {
@@ -317,8 +311,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_commit_pair(smem_u32(drain));
       mbar_wait_drain(smem_u32(drain), 0);
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale-ring producer (both CTAs)
+    // Its own thread, so that a slot the scale warps have not yet freed never
+    // holds up the A/B stages.
+    if (lane == 0) {
+      uint32_t ksf = 0;
+      while (ksf < total_ks && issue_sf(ksf)) ++ksf;
+      // no scale copy may still be landing when shared memory goes away
+      const uint32_t sf_first = ksf > static_cast<uint32_t>(C::SF_STAGES) ? ksf - C::SF_STAGES : 0u;
+      for (uint32_t k = sf_first; k < ksf; ++k)
+        mbar_wait_drain(smem_u32(&sf_full[k % C::SF_STAGES]), (k / C::SF_STAGES) & 1);
+    }
   } else if (warp < C::SF_WARP0) {
-    // spare warps
+    // spare warp
   } else if (warp >= C::EPI_WARP0) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     regs_grow_to<C::REGS_EPI>();
