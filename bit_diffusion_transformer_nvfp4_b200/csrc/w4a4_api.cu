@@ -37,6 +37,12 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// The main pair configuration: 256 x 256 tiles, six 32 KB A/B stages, a
+// three-slot scale ring, one epilogue staging buffer per warp, no alignment
+// slack (the kernel checks that the dynamic shared memory base is 1024-byte
+// aligned and reports W4A4_ERR_DEVICE_LAYOUT otherwise): 226 KB.
+using PairMain = Gemm2Cfg<256, 6, 3, 1, false>;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -85,7 +91,7 @@ int device_setup(DeviceInfo** out) {
              cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm_kernel<G192>, cudaFuncAttributeMaxDynamicSharedMemorySize, G192::SMEM) ==
              cudaSuccess;
-  using P256 = Gemm2Cfg<256, 5>;
+  using P256 = PairMain;
   using P192 = Gemm2Cfg<192, 5>;
   using P64 = Gemm2Cfg<64, 6>;
   attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P64>, cudaFuncAttributeMaxDynamicSharedMemorySize, P64::SMEM) ==
@@ -601,7 +607,7 @@ static int gemm_dispatch(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x
   // that gives at most two tiles per pair, so a small layer streams its
   // weight through many SMs; else single-CTA 128 x 192 / 128 x 256 tiles.
   if (M > 128)
-    return launch_gemm_pair<Gemm2Cfg<256, 5>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
+    return launch_gemm_pair<PairMain>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
                                               next_inv_s, next_amax, s, dev);
   if (ceil_div(N, 64) <= static_cast<int64_t>(dev->num_sms))
     return launch_gemm_pair<Gemm2Cfg<64, 6>>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
