@@ -620,6 +620,13 @@ __global__ void sf_to_rowmajor_kernel(const uint8_t* __restrict__ atoms, int64_t
 constexpr int kFusedMaxChunks = 12;
 constexpr int kFusedL1Ring = 7;  // L1t tiles in flight: as many as fit beside the resident X
 constexpr int kFusedSlicesForSpread = 16;
+// Grid barrier words in the workspace (32-bit word offsets, each on its own
+// 128-byte line): the launch generation, two arrival counters and two
+// tensor-maximum words (one of each per generation parity).
+constexpr int kBarGen = 0;
+constexpr int kBarCount = 32;   // + 32 * parity
+constexpr int kBarAmax = 96;    // + 32 * parity
+constexpr int kBarWords = 160;
 
 struct FusedQuantSmem {
   static constexpr int kXBytes = kFusedMaxChunks * kQRows * kQChunk * 2;   // 192 KB
@@ -650,6 +657,24 @@ static_assert(kFComputeWarps * 32 >= 256, "one thread per scale code fills the m
 
 static_assert(kFUWarp0 % 4 == 0 && kFThreads == 32 * (kFUWarp0 + 4), "lane quarters");
 
+// The grid barrier.  Every launch reads the generation G and uses the
+// counter and maximum word of parity G & 1: each CTA folds its maximum into
+// the word (atomic max; non-negative floats order as their bit patterns),
+// then adds one to the counter with release semantics, and waits until the
+// counter shows every CTA.  Block 0 then clears the other parity's two words
+// for the next launch and advances G; the words of this launch's parity stay
+// as they are until the launch after next clears them, so no CTA waits for a
+// second round of atomics to learn that everyone has read the maximum.
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Bounded spin until a global counter reaches ``target``; false on timeout
 // (then the abort flag and the device status are set).
 __device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target, volatile int* abort, int* status) {
@@ -668,7 +693,8 @@ __device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target,
 
 __global__ void __launch_bounds__(kFThreads, 1)
     quant_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
-                       const __grid_constant__ CUtensorMap tm_q, const QuantParams p, unsigned* grid_sync) {
+                       const __grid_constant__ CUtensorMap tm_q, const QuantParams p, unsigned* tickets,
+                       unsigned* barrier) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
@@ -683,14 +709,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(tmem_slot + 2);  // kFComputeWarps floats
   float* t_shared = reinterpret_cast<float*>(tmem_slot + 2 + kFComputeWarps);
-  // Zero at rest.  counter: CTAs that have contributed their maximum (first
-  // gridDim.x increments), then CTAs that have read the result (second
-  // gridDim.x); the last reader clears it and the amax word.  tickets[rb]:
-  // slices of the row block whose partial U is out, then slices that have
-  // seen them all; the last clears it.
-  unsigned* counter = grid_sync;
-  unsigned* amax_bits = grid_sync + 1; // running max of the CTA maxima (non-negative floats order as bits)
-  unsigned* tickets = grid_sync + 2;
+  unsigned* gen_shared = tmem_slot + 3 + kFComputeWarps;
+  // tickets[rb] (zero at rest): slices of the row block whose partial U is
+  // out, then slices that have seen them all; the last clears it.
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -727,6 +748,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   // set-up above may overlap the previous kernel (programmatic launch);
   // nothing below may touch memory before it has completed
   grid_dependency_wait();
+  if (tid == 0) *gen_shared = ld_relaxed_gpu(barrier + kBarGen);
 
   float bmax[4 * kFChunksPerThread];  // compute threads: block maxima of their row
   const int r = tid & (kQRows - 1);
@@ -905,16 +927,21 @@ __global__ void __launch_bounds__(kFThreads, 1)
       float a = red[0];
 #pragma unroll
       for (int w = 1; w < kFComputeWarps; ++w) a = fmaxf(a, red[w]);
+      const unsigned g = *gen_shared;
+      unsigned* count = barrier + kBarCount + 32 * (g & 1u);
+      unsigned* amax_bits = barrier + kBarAmax + 32 * (g & 1u);
       atomicMax(amax_bits, __float_as_uint(a));
-      red_release_add(counter, 1u);
-      if (spin_until(counter, gridDim.x, abort_flag, p.status)) {
-        const float t = tensor_scale_from(__uint_as_float(ld_acquire_gpu(amax_bits)));
+      red_release_add(count, 1u);  // orders the maximum before the arrival
+      if (spin_until(count, gridDim.x, abort_flag, p.status)) {
+        const float t = tensor_scale_from(__uint_as_float(ld_relaxed_gpu(amax_bits)));
         *t_shared = t;
         if (blockIdx.x == 0) *p.t_out = t;
-        if (atom_acq_rel_add(counter, 1u) == 2u * gridDim.x - 1u) {
-          *amax_bits = 0u;  // every CTA has read it
-          *counter = 0u;
-        }
+      }
+      if (blockIdx.x == 0) {
+        // every CTA has read G (its arrival used it), also after a timeout
+        st_relaxed_gpu(barrier + kBarCount + 32 * ((g + 1u) & 1u), 0u);
+        st_relaxed_gpu(barrier + kBarAmax + 32 * ((g + 1u) & 1u), 0u);
+        st_relaxed_gpu(barrier + kBarGen, g + 1u);
       }
     }
     named_bar_sync(1, 32 * kFComputeWarps);
@@ -923,8 +950,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
     if (*abort_flag) return;
 
     // ------------------------------------------------------ phase B: scales and codes
-    // The code multiplier 1/(dec(e) t) of every scale code, once per CTA.
-    if (tid < 256) rq_tab[tid] = __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(tid)).y, t));
+    // The code multiplier 1/(dec(e) t) of every scale code a block can get
+    // (1..126: non-negative, saturated at 448), once per CTA.  Code 0 leaves
+    // the block's codes +0 (its entry is never used); skipping it and the
+    // codes above 126 keeps every reciprocal on the fast path (with them,
+    // the table took 0.55 us instead of 0.16).
+    if (tid < 256)
+      rq_tab[tid] = (tid >= 1 && tid <= 126)
+                        ? __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(tid)).y, t))
+                        : 0.0f;
     named_bar_sync(1, 32 * kFComputeWarps);
     const float rt = __frcp_rn(t);
     // Codes leave through TMA stores of the warp's 32 rows x 32 bytes, staged
@@ -950,19 +984,19 @@ __global__ void __launch_bounds__(kFThreads, 1)
           for (int q = 0; q < 2; ++q) {
             const int b = 2 * h + q;
             const uint32_t e = (e2 >> (8 * q)) & 0xFFu;
-            cw[2 * b] = cw[2 * b + 1] = 0u;
-            if (e != 0u) {  // a zero scale leaves the block's codes +0
-              const float rq = rq_tab[e];
+            // a zero scale leaves the block's codes +0: computed anyway and
+            // masked, so that no branch keeps the loads from moving up
+            const float rq = rq_tab[e];
 #pragma unroll
-              for (int uu = 0; uu < 2; ++uu) {
-                float v[8];
-                load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
-                mul2_rn(v[0], v[1], v[0], v[1], rq, rq);
-                mul2_rn(v[2], v[3], v[2], v[3], rq, rq);
-                mul2_rn(v[4], v[5], v[4], v[5], rq, rq);
-                mul2_rn(v[6], v[7], v[6], v[7], rq, rq);
-                cw[2 * b + uu] = cvt_e2m1x8(v);
-              }
+            for (int uu = 0; uu < 2; ++uu) {
+              float v[8];
+              load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
+              mul2_rn(v[0], v[1], v[0], v[1], rq, rq);
+              mul2_rn(v[2], v[3], v[2], v[3], rq, rq);
+              mul2_rn(v[4], v[5], v[4], v[5], rq, rq);
+              mul2_rn(v[6], v[7], v[6], v[7], rq, rq);
+              const uint32_t c8 = cvt_e2m1x8(v);
+              cw[2 * b + uu] = e != 0u ? c8 : 0u;
             }
           }
         }

@@ -132,7 +132,7 @@ struct QuantPlan {
   int64_t row_blocks = 0;
   int chunks = 0, splits = 0, chunks_per_split = 0;
   int upart_slices = 0;  // K slices the low-rank partial buffer holds
-  size_t off_partials = 0, off_tickets = 0, off_upart = 0, bytes = 0;
+  size_t off_partials = 0, off_tickets = 0, off_barrier = 0, off_upart = 0, bytes = 0;
 };
 
 // SM count the work split and the workspace size assume (B200); on another
@@ -180,10 +180,11 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
   const int slices_max = std::max(q.splits, fused_splits(q.row_blocks, q.chunks, kPlanSms));
   q.off_partials = 0;
   q.off_tickets = round256(sizeof(float) * kAmaxMaxBlocks);
-  // counters, zero at rest (each kernel clears what it used): the two-pass
-  // path's per-row-block tickets, or the single-pass path's grid-barrier
-  // counter, tensor-amax word and per-row-block tickets
-  q.off_upart = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks + 2));
+  // per-row-block tickets of the low-rank sums, zero at rest (each kernel
+  // clears the ones it used); then the single-pass path's grid barrier
+  // (launch generation, counters and maximum words per generation parity)
+  q.off_barrier = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks));
+  q.off_upart = q.off_barrier + round256(sizeof(unsigned) * kBarWords);
   q.upart_slices = slices_max;
   const size_t upart = r > 0 ? sizeof(float) * static_cast<size_t>(slices_max) * q.row_blocks * kQRows * 32 : 0;
   q.bytes = q.off_upart + round256(upart);
@@ -207,9 +208,10 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   if (cps > kFusedMaxChunks || rb * splits > dev->num_sms || splits > plan.upart_slices) return -1;
 
   uint8_t* w = static_cast<uint8_t*>(ws);
-  // grid-barrier counter, tensor-amax bits, one ticket per row block (zero at
-  // rest: the kernel clears them before it ends)
-  unsigned* grid_sync = reinterpret_cast<unsigned*>(w + plan.off_tickets);
+  // one ticket per row block (zero at rest: the kernel clears them before it
+  // ends) and the grid barrier's words
+  unsigned* tickets = reinterpret_cast<unsigned*>(w + plan.off_tickets);
+  unsigned* barrier = reinterpret_cast<unsigned*>(w + plan.off_barrier);
   CUtensorMap tm_x, tm_l1;
   if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(ld) * 2, 64u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -257,10 +259,10 @@ int launch_quant_fused(const __nv_bfloat16* X, int64_t M, int64_t K, int64_t ld,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, grid_sync) == cudaSuccess) return W4A4_OK;
+  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, tickets, barrier) == cudaSuccess) return W4A4_OK;
   cudaGetLastError();
   cfg.numAttrs = 1;  // without the programmatic attribute
-  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, grid_sync) == cudaSuccess) return W4A4_OK;
+  if (cudaLaunchKernelEx(&cfg, quant_fused_kernel, tm_x, tm_l1, tm_q, p, tickets, barrier) == cudaSuccess) return W4A4_OK;
   cudaGetLastError();
   return -1;  // not co-resident on this device: fall back
 }

@@ -97,11 +97,12 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
  *
  * Workspace contract (every entry point that takes a workspace): zero the
  * whole workspace once before its first use (cudaMemset, torch.zeros).  The
- * counters in it are zero at rest: each call clears the ones it used before
- * its last kernel ends, so no clearing is needed between calls, whatever
- * their sizes.  After a call reports a device error (w4a4_device_status),
- * zero the workspace again.  Calls that overlap on the GPU must not share a
- * workspace. */
+ * synchronisation words in it stay valid from call to call (counters are
+ * cleared by the call that used them; the single-pass grid barrier keeps a
+ * launch generation that every call advances), so no clearing is needed
+ * between calls, whatever their sizes.  After a call reports a device error
+ * (w4a4_device_status), zero the workspace again.  Calls that overlap on the
+ * GPU must not share a workspace. */
 size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r);
 
 /* Workspace bytes needed by w4a4_linear: the quantisation workspace plus the

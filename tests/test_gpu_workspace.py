@@ -1,9 +1,9 @@
-"""Workspace counters are zero at rest.
+"""One workspace, zeroed once, serves any sequence of calls.
 
-The quantiser's grid barrier, its tensor-amax word and the per-row-block
-tickets of the low-rank sums live in the caller's workspace; every call
-clears what it used before its last kernel ends, so one workspace, zeroed
-once, serves any sequence of calls.  Here one shared workspace runs the
+The quantiser's per-row-block tickets of the low-rank sums (zero at rest:
+every call clears what it used) and the single-pass grid barrier (a launch
+generation that every call advances, and one tagged slot per CTA) live in
+the caller's workspace.  Here one shared workspace runs the
 single-pass cooperative path, the two-pass path (an activation too large to
 be co-resident) and the quantise-with-given-amax path, in an order that
 changes the grid size and the number of row blocks between calls; every
