@@ -967,37 +967,48 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // drain barrier has fired (long before this point).
     if (lr && !mbar_wait(smem_u32(drain), 0, abort_flag, p.status)) return;
     if (lane == 0) tma_prefetch_desc(&tm_q);
+    // Every scale byte of the thread first (sixteen independent chains; the
+    // scale words go out at once) with its code multiplier kept in a
+    // register, then the codes chunk by chunk: no code waits on a table
+    // lookup.
+    uint32_t e4[kFChunksPerThread];
+    float rq[4 * kFChunksPerThread];
+#pragma unroll
+    for (int i = 0; i < kFChunksPerThread; ++i) {
+      // two blocks' scale bytes per conversion; byte b = block b
+      const uint32_t lo = cvt_e4m3x2(div6(__fmul_rn(bmax[4 * i + 1], rt)), div6(__fmul_rn(bmax[4 * i], rt)));
+      const uint32_t hi = cvt_e4m3x2(div6(__fmul_rn(bmax[4 * i + 3], rt)), div6(__fmul_rn(bmax[4 * i + 2], rt)));
+      e4[i] = (lo & 0xFFFFu) | (hi << 16);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) rq[4 * i + b] = rq_tab[(e4[i] >> (8 * b)) & 0xFFu];
+      const int c = grp + kFGroups * i;
+      if (c < n) {
+        const int64_t atom = static_cast<int64_t>(rb) * chunks + kc0 + c;
+        *reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (r & 31) * 16 + (r >> 5) * 4) = e4[i];
+      }
+    }
 #pragma unroll
     for (int i = 0; i < kFChunksPerThread; ++i) {
       const int c = grp + kFGroups * i;
       if (c < n) {
         const int kc = kc0 + c;
-        uint32_t e4 = 0u;
         uint32_t cw[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // two blocks' scale bytes in one conversion; byte 0 = block 2h
-          const uint32_t e2 = cvt_e4m3x2(div6(__fmul_rn(bmax[4 * i + 2 * h + 1], rt)),
-                                         div6(__fmul_rn(bmax[4 * i + 2 * h], rt))) & 0xFFFFu;
-          e4 |= e2 << (16 * h);
+        for (int b = 0; b < 4; ++b) {
+          // a zero scale leaves the block's codes +0 (computed anyway and
+          // masked: no branch keeps the loads from moving up)
+          const bool zero = ((e4[i] >> (8 * b)) & 0xFFu) == 0u;
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int b = 2 * h + q;
-            const uint32_t e = (e2 >> (8 * q)) & 0xFFu;
-            // a zero scale leaves the block's codes +0: computed anyway and
-            // masked, so that no branch keeps the loads from moving up
-            const float rq = rq_tab[e];
-#pragma unroll
-            for (int uu = 0; uu < 2; ++uu) {
-              float v[8];
-              load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
-              mul2_rn(v[0], v[1], v[0], v[1], rq, rq);
-              mul2_rn(v[2], v[3], v[2], v[3], rq, rq);
-              mul2_rn(v[4], v[5], v[4], v[5], rq, rq);
-              mul2_rn(v[6], v[7], v[6], v[7], rq, rq);
-              const uint32_t c8 = cvt_e2m1x8(v);
-              cw[2 * b + uu] = e != 0u ? c8 : 0u;
-            }
+          for (int uu = 0; uu < 2; ++uu) {
+            float v[8];
+            load_unit<__nv_bfloat16>(xs + c * kQRows * kQChunk * 2, invs + c * kQChunk, has_inv, r, 2 * b + uu, v);
+            const float m = rq[4 * i + b];
+            mul2_rn(v[0], v[1], v[0], v[1], m, m);
+            mul2_rn(v[2], v[3], v[2], v[3], m, m);
+            mul2_rn(v[4], v[5], v[4], v[5], m, m);
+            mul2_rn(v[6], v[7], v[6], v[7], m, m);
+            const uint32_t c8 = cvt_e2m1x8(v);
+            cw[2 * b + uu] = zero ? 0u : c8;
           }
         }
         // every lane has read its rows of the chunk: stage this warp's codes
@@ -1017,8 +1028,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
           tma_store_2d(&tm_q, smem_u32(cb), kc * 32, rb * kQRows + (warp & 3) * 32);
           bulk_commit_group();
         }
-        const int64_t atom = static_cast<int64_t>(rb) * chunks + kc;
-        *reinterpret_cast<uint32_t*>(p.sf + atom * 512 + (r & 31) * 16 + (r >> 5) * 4) = e4;
       }
     }
     // the code stores have landed before the CTA ends
