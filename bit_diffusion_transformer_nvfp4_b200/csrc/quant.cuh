@@ -1,26 +1,33 @@
 // quant.cuh -- NVFP4 quantisation kernels.
 //
-//   amax_kernel   pass 1: A = max |x * inv_s| over the tensor.  Grid-stride,
-//                 16-byte loads, warp-shuffle + shared-memory block max, one
-//                 partial maximum per CTA (no atomics, so the result is
-//                 deterministic).
-//   quant_kernel  pass 2: one CTA per (128-row block, K slice).  TMA streams
-//                 128 x 64 tiles of the source through a 4-stage mbarrier
-//                 ring (128-byte swizzle); thread t owns row t of the tile,
-//                 so the four 16-element blocks of a 64-wide chunk are
-//                 reduced without shuffles and its four scale bytes form one
-//                 32-bit word of the SF atom.  When a low-rank factor is
-//                 given, one elected thread feeds the same shared-memory
-//                 tile to tcgen05.mma (kind::f16, M=128, N=r=32) so that
-//                 U = X L1 accumulates in TMEM; each K slice writes its fp32
-//                 partial, and the last slice of a row block (ticket counter)
-//                 sums the partials in slice order, scales by 1/(t_x t_w) and
-//                 writes the bf16 hi/lo pair.
+//   amax_kernel         A = max |x * inv_s| over the tensor.  Grid-stride,
+//                       16-byte loads, warp-shuffle + shared-memory block
+//                       max, one partial maximum per CTA (no atomics, so the
+//                       result is deterministic).
+//   quant_kernel        the streaming quantise pass, tensor amax known:
+//                       persistent, one CTA per SM walking (128-row block,
+//                       K slice) work items; TMA streams 128 x 64 tiles of
+//                       the source through one mbarrier ring (128-byte
+//                       swizzle); thread t owns row t of the tile, so the
+//                       four 16-element blocks of a 64-wide chunk are reduced
+//                       without shuffles and its four scale bytes form one
+//                       32-bit word of the SF atom.  With a low-rank factor,
+//                       one elected thread feeds the same tiles to
+//                       tcgen05.mma (kind::f16, M=128, N=r) so that U = X L1
+//                       accumulates in TMEM; each K slice writes its fp32
+//                       partial, and the last slice of a row block (ticket
+//                       counter) sums the partials in slice order, scales by
+//                       1/(t_x t_w) and writes the bf16 hi/lo pair.
+//   quant_fused_kernel  the single pass: every tile of the activation stays
+//                       resident in shared memory while a grid barrier
+//                       reduces the tensor amax, then the same quantisation.
 //
-// Counters in the workspace (grid barrier, tensor amax word, per-row-block
-// tickets) are zero at rest: every kernel that uses one returns it to zero
-// before it ends (the last participant to read it clears it), so a call needs
-// no memset as long as the workspace was zeroed once before its first use.
+// Synchronisation words in the workspace: the per-row-block tickets are zero
+// at rest (the last participant to read one clears it before its kernel
+// ends); the single-pass grid barrier keeps a launch generation and, per
+// generation parity, an arrival counter and a maximum word, the other
+// parity's pair being cleared one launch ahead.  A call therefore needs no
+// memset as long as the workspace was zeroed once before its first use.
 //
 // The quantiser follows the NVFP4 arithmetic stated in include/w4a4.h; every
 // rounding step is an explicit correctly rounded fp32 intrinsic so that codes
