@@ -182,8 +182,9 @@ def _u8(n, device):
 
 
 def new_workspace(nbytes, device):
-    """A workspace for the entry points that take one: zeroed once, as the
-    library's counters must start at zero (every call leaves them zero)."""
+    """A workspace for the entry points that take one, zeroed once: the
+    library's synchronisation words start from zeros and every call leaves
+    them valid for the next (zero it again only after a device error)."""
     return torch.zeros(max(16, nbytes), dtype=torch.uint8, device=device)
 
 
