@@ -840,8 +840,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (tid == 32 * kFUWarp0) red_release_add(tickets + rb, 1u);
       // ---------------------------------------------------- wait for the tensor scale
       named_bar_sync(2, kFThreads);
-      if (!*abort_flag) {
-        if (tid == 32 * kFUWarp0 &&
+      {
+        // the four U warps meet at barrier 3 whatever the abort flag says
+        if (tid == 32 * kFUWarp0 && !*abort_flag &&
             spin_until(tickets + rb, static_cast<unsigned>(p.splits), abort_flag, p.status) &&
             atom_acq_rel_add(tickets + rb, 1u) == 2u * static_cast<unsigned>(p.splits) - 1u)
           tickets[rb] = 0u;  // every slice has passed
@@ -954,7 +955,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
     named_bar_sync(1, 32 * kFComputeWarps);
     if (lr) named_bar_arrive(2, kFThreads);  // the tensor scale is out for the U warps
     const float t = *t_shared;
-    if (*abort_flag) return;
 
     // ------------------------------------------------------ phase B: scales and codes
     // The code multiplier 1/(dec(e) t) of every scale code a block can get
@@ -967,6 +967,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
                         ? __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(tid)).y, t))
                         : 0.0f;
     named_bar_sync(1, 32 * kFComputeWarps);
+    // after the last named barrier of the compute warps: a warp that leaves
+    // here never leaves another waiting at a barrier
+    if (*abort_flag) return;
     const float rt = __frcp_rn(t);
     // Codes leave through TMA stores of the warp's 32 rows x 32 bytes, staged
     // in the first kilobyte of the warp's own rows of the chunk it has just
