@@ -76,3 +76,27 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
 
     assert bench.run_reference(Args()) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
+    """Rank 0 times the oracle on a small sample of the same workload and
+    prints one line with the main arm's metric, the reference marker, its
+    own CPU-baseline description and a zero-copy end-to-end figure."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+
+    class Args:
+        steps, warmup, ref_rows, ref_cols = 1, 3, 16, 32
+
+    bench.run_reference(Args())
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOPS"
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 3
+    assert d["config"]["workload"] == bench.WORKLOAD["workload"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and "16 of" in cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
