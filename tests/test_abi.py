@@ -85,6 +85,34 @@ def test_host_validation_before_any_launch(so):
     assert pw(P, 5, 128, 512, 512, P, P, P, P, big, None) == -8                               # dtype
 
 
+
+def test_host_validation_linear_and_amax_entries(so):
+    """The whole-path and given/next-amax entry points reject bad arguments on
+    the host, in the documented order, before touching a GPU."""
+    P = 1 << 20  # aligned fake device address, never dereferenced
+    big = 1 << 30
+    lin = so.w4a4_linear
+    #        X  M    N    K    Wq Wsf t_w inv_s L1t L2t r   bias  epi Y  ws  ws_bytes stream
+    assert lin(P, 128, 100, 512, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -2   # N % 8
+    assert lin(P, 128, 128, 500, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -2   # K % 256
+    assert lin(P, 128, 128, 512, P, P, P, None, P, P, 24, None, 0, P, P, big, None) == -2   # rank
+    assert lin(P, 128, 128, 512, P, P, P, None, P, P, 32, None, 7, P, P, big, None) == -8   # epilogue
+    assert lin(None, 128, 128, 512, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -1  # NULL X
+    assert lin(P, 128, 128, 512, P, P, P, None, None, P, 32, None, 0, P, P, big, None) == -1  # rank 32, no L1t
+    assert lin(P, 128, 128, 512, P, P, P, None, P, P, 32, None, 0, P, P, 16, None) == -5    # workspace size
+    assert lin(P, 128, 128, 512, P, P, P, None, P, P, 32, None, 0, P, P + 2, big, None) == -3  # workspace align
+    qa = so.nvfp4_quantize_act_with_amax
+    #        X  M    K    ldx inv_s L1t r  t_w  amax   Xq Xsf t_x U     ws  ws_bytes stream
+    assert qa(P, 128, 512, 512, None, None, 0, None, None, P, P, P, None, P, big, None) == -1  # no amax
+    assert qa(P, 128, 512, 512, None, None, 0, None, P + 2, P, P, P, None, P, big, None) == -3  # amax align
+    assert qa(P, 128, 500, 512, None, None, 0, None, P, P, P, P, None, P, big, None) == -2      # K % 256
+    gn = so.w4a4_gemm_next_amax
+    #       Xq Xsf t_x U     M    N    K    Wq Wsf t_w L2t  r  bias  epi Y  ldy  inv_s  amax   stream
+    assert gn(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 128, None, None, None) == -1
+    assert gn(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 128, P + 4, P, None) == -3
+    assert gn(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 128, None, P + 2, None) == -3
+    assert gn(P, P, P, None, 128, 100, 512, P, P, P, None, 0, None, 0, P, 100, None, P, None) == -2
+
 def test_empty_problems_are_noops(so):
     """M == 0 (N == 0 for packing) with valid sizes: W4A4_OK at once, with
     NULL buffers, no device needed; invalid sizes still fail."""
