@@ -337,3 +337,41 @@ def test_bf16_rounding_against_library():
     ref = torch.tensor(v).to(torch.bfloat16).to(torch.float32).numpy()
     np.testing.assert_array_equal(prep.to_bf16_values(v), ref)
     np.testing.assert_array_equal(bf16_round(v), ref)
+
+
+# ---------------------------------------------------------------- parity checkers
+# Every Y verdict rests on these two functions, so each is pinned to values
+# worked out by hand, on cases where the plausible mistakes (normalising by
+# the tested result instead of the reference, reducing over columns or over
+# the whole matrix instead of per row) give a different number.
+
+def test_rel_frobenius_by_hand():
+    ref = np.array([[1.0, 10.0], [6.0, 8.0]])
+    test = np.array([[1.0, 10.0], [6.0, 4.0]])
+    # |test - ref|_F = 4, |ref|_F = sqrt(1 + 100 + 36 + 64) = sqrt(201)
+    assert linear.rel_frobenius(test, ref) == pytest.approx(4.0 / np.sqrt(201.0), rel=1e-15)
+    # normalising by |test|_F = sqrt(153) would give 0.3234 instead of 0.2821
+    assert abs(linear.rel_frobenius(test, ref) - 4.0 / np.sqrt(153.0)) > 0.04
+    # a 3-4-5 case: the difference (0.3, 0.4) against (3, 4) is exactly 0.1
+    assert linear.rel_frobenius(np.array([[3.3, 4.4]]), np.array([[3.0, 4.0]])) == pytest.approx(0.1, rel=1e-12)
+    assert linear.rel_frobenius(ref, ref) == 0.0
+    # an all-zero reference falls back to the absolute norm of the difference
+    assert linear.rel_frobenius(np.array([[0.0, 3.0], [4.0, 0.0]]), np.zeros((2, 2))) == 5.0
+
+
+def test_row_maxabs_ratio_by_hand():
+    ref = np.array([[1.0, 10.0], [6.0, 8.0]])
+    test = np.array([[1.0, 10.0], [6.0, 4.0]])
+    # row 0: 0 / 10; row 1: |4 - 8| / max(6, 8) = 0.5
+    assert linear.row_maxabs_ratio(test, ref) == 0.5
+    # over columns it would be 0.4 (4 / 10), over the whole matrix 0.4, and
+    # against the tested row's maximum 4 / 6
+    assert linear.row_maxabs_ratio(test.T, ref.T) == 0.4
+    # a zero reference row is compared in absolute terms
+    assert linear.row_maxabs_ratio(np.array([[0.0, 1e-3], [2.0, 2.0]]),
+                                   np.array([[0.0, 0.0], [2.0, 2.0]])) == 1e-3
+    # the largest row ratio wins, whatever the row order
+    a = np.array([[10.0, 0.0], [1.0, 0.0], [4.0, 4.0]])
+    b = a + np.array([[1.0, 0.0], [0.5, 0.0], [0.0, -1.0]])
+    assert linear.row_maxabs_ratio(b, a) == 0.5
+    assert linear.row_maxabs_ratio(b[::-1], a[::-1]) == 0.5
