@@ -20,7 +20,8 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_pack_weight", "w4a4_gemm", "w4a4_linear", "w4a4_device_status",
     "w4a4_status_string", "EPI_NONE", "EPI_GELU_TANH", "SRC_BF16", "SRC_F32",
     "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
-    "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor",
+    "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor", "w4a4_set_wait_bound",
+    "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -47,7 +48,9 @@ _SIG = {
                                        _c.c_int, _P, _I64, _P, _P, _P]),
     "w4a4_linear": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _c.c_int, _P, _c.c_int, _P,
                                _P, _c.c_size_t, _P]),
+    "nvfp4_quantize_act_noalloc": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P, _P]),
     "w4a4_device_status": (_c.c_int, [_c.POINTER(_c.c_int), _c.c_int]),
+    "w4a4_set_wait_bound": (_c.c_int, [_I64]),
     "nvfp4_sf_to_rowmajor": (_c.c_int, [_P, _I64, _I64, _P, _P]),
     "w4a4_status_string": (_c.c_char_p, [_c.c_int]),
 }
@@ -165,6 +168,17 @@ def sf_rowmajor(sf_atoms: torch.Tensor, rows: int, K: int, stream=None) -> torch
     out = torch.empty(rows, K // 16, dtype=torch.uint8, device=sf_atoms.device)
     nvfp4_sf_to_rowmajor(sf_atoms, rows, K, out, stream)
     return out
+
+
+def w4a4_set_wait_bound(cycles: int = 0) -> None:
+    """Device-side waits give up after ``cycles`` SM clock cycles (0: the default)."""
+    _check("w4a4_set_wait_bound", lib().w4a4_set_wait_bound(cycles))
+
+
+def nvfp4_quantize_act_noalloc(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, stream=None):
+    _check("nvfp4_quantize_act_noalloc", lib().nvfp4_quantize_act_noalloc(
+        _ptr(X), M, K, ldx, _ptr(inv_s), _ptr(L1t), r, _ptr(t_w), _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U),
+        _stream(stream)))
 
 
 def w4a4_device_status(reset: bool = False) -> int:

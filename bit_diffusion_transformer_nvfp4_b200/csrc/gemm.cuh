@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int m_tiles = (p.M + C::BM - 1) / C::BM;
   const int n_tiles = (p.N + BN - 1) / BN;
   const int total = m_tiles * n_tiles;
-  const int nkb = p.K / C::BK;
+  const int nkb = (p.K + C::BK - 1) / C::BK;  // the last K step may be partial: TMA fills zeros
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int m_tiles = (p.M + 2 * C::BM - 1) / (2 * C::BM);
   const int n_tiles = (p.N + BN - 1) / BN;
   const int total = m_tiles * n_tiles;
-  const int nkb = p.K / C::BK;
+  const int nkb = (p.K + C::BK - 1) / C::BK;  // the last K step may be partial: TMA fills zeros
   const int pair = blockIdx.x >> 1;
   const int pairs = gridDim.x >> 1;
   // K steps (with scales) this pair runs: every tile pair, pair+pairs, ...

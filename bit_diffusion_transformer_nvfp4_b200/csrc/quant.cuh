@@ -688,7 +688,7 @@ __device__ __forceinline__ bool spin_until(const unsigned* ctr, unsigned target,
   const long long start = clock64();
   while (ld_acquire_gpu(ctr) < target) {
     if (*abort) return false;
-    if (clock64() - start > kWaitBoundCycles) {
+    if (clock64() - start > c_wait_bound_cycles) {
       *abort = 1;
       if (status) atomicExch(status, kStatusTimeout);
       return false;
@@ -946,7 +946,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (blockIdx.x == 0) *p.t_out = t;
       }
       if (blockIdx.x == 0) {
-        // every CTA has read G (its arrival used it), also after a timeout
+        // Once the counter shows every CTA, every CTA has read G (its arrival
+        // used it).  After a timeout some CTA may not have arrived yet and
+        // may still arrive on this parity: the words are then left
+        // inconsistent, the status word says so, and the caller zeroes the
+        // workspace before its next use.
         st_relaxed_gpu(barrier + kBarCount + 32 * ((g + 1u) & 1u), 0u);
         st_relaxed_gpu(barrier + kBarAmax + 32 * ((g + 1u) & 1u), 0u);
         st_relaxed_gpu(barrier + kBarGen, g + 1u);

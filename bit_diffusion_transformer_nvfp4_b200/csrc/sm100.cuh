@@ -16,8 +16,11 @@ namespace w4a4 {
 constexpr int kStatusTimeout = -7;
 constexpr int kStatusMisaligned = -10;
 
-// A wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz).
-constexpr long long kWaitBoundCycles = 4000000000LL;
+// A wait gives up after this many SM clock cycles: by default 4e9, about
+// 2 s at 1.9 GHz.  Set per device by w4a4_set_wait_bound (host code writes
+// the constant bank between launches).
+constexpr long long kDefaultWaitBoundCycles = 4000000000LL;
+__constant__ long long c_wait_bound_cycles = kDefaultWaitBoundCycles;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -75,7 +78,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - start > kWaitBoundCycles) {
+    if (clock64() - start > c_wait_bound_cycles) {
       *abort = 1;
       if (status) atomicExch(status, kStatusTimeout);
       return false;
@@ -87,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const long long start = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - start > kWaitBoundCycles / 8) return;
+    if (clock64() - start > c_wait_bound_cycles / 8) return;
   }
 }
 

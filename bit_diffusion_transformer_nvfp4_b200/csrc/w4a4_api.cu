@@ -139,6 +139,16 @@ struct QuantPlan {
 // count the kernels stay correct, only the balance changes.
 constexpr int kPlanSms = 148;
 
+// Workspace layout (byte offsets; documented in include/w4a4.h).
+constexpr size_t kWsBarrierOff = sizeof(float) * kAmaxMaxBlocks;                   // 4096
+constexpr size_t kWsTicketsOff = kWsBarrierOff + 1024;                              // 160 words on 128-byte lines
+constexpr int64_t kMaxTicketRowBlocks = W4A4_MAX_LOWRANK_ROWS / kQRows;             // 32768
+constexpr size_t kWsUpartOff = kWsTicketsOff + sizeof(unsigned) * kMaxTicketRowBlocks;
+static_assert(sizeof(unsigned) * kBarWords <= 1024, "barrier words fit their slot");
+static_assert(kWsBarrierOff == W4A4_WS_BARRIER_OFFSET && kWsTicketsOff == W4A4_WS_TICKETS_OFFSET &&
+                  kWsUpartOff == W4A4_WS_UPART_OFFSET,
+              "layout constants of the header");
+
 // K-slice count of the single-pass path (its tile set is co-resident: one CTA
 // per (row block, slice), at most kFusedMaxChunks chunks each).
 int fused_splits(int64_t row_blocks, int chunks, int64_t sms) {
@@ -178,20 +188,26 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
     }
   }
   const int slices_max = std::max(q.splits, fused_splits(q.row_blocks, q.chunks, kPlanSms));
+  // Fixed layout, the same for every M, K and r (so that one workspace
+  // serves any sequence of calls): amax partial maxima; the single-pass
+  // grid barrier (launch generation, counters and maximum words per
+  // generation parity); one low-rank ticket per 128-row block up to
+  // kMaxTicketRowBlocks (zero at rest: each kernel clears the ones it used);
+  // then the fp32 low-rank partial sums, whose size alone depends on M.
   q.off_partials = 0;
-  q.off_tickets = round256(sizeof(float) * kAmaxMaxBlocks);
-  // per-row-block tickets of the low-rank sums, zero at rest (each kernel
-  // clears the ones it used); then the single-pass path's grid barrier
-  // (launch generation, counters and maximum words per generation parity)
-  q.off_barrier = q.off_tickets + round256(sizeof(int) * static_cast<size_t>(q.row_blocks));
-  q.off_upart = q.off_barrier + round256(sizeof(unsigned) * kBarWords);
+  q.off_barrier = kWsBarrierOff;
+  q.off_tickets = kWsTicketsOff;
+  q.off_upart = kWsUpartOff;
   q.upart_slices = slices_max;
   const size_t upart = r > 0 ? sizeof(float) * static_cast<size_t>(slices_max) * q.row_blocks * kQRows * 32 : 0;
   q.bytes = q.off_upart + round256(upart);
   return q;
 }
 
-bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0 && K <= (int64_t(1) << 30); }
+bool valid_k(int64_t K) { return K >= 64 && K % 64 == 0 && K <= (int64_t(1) << 30); }
+
+// Rows the per-row-block low-rank counters of a workspace cover.
+bool valid_lowrank_rows(int64_t M, int r) { return r == 0 || M <= W4A4_MAX_LOWRANK_ROWS; }
 
 // Single-pass activation quantisation: every (row block, K slice) tile must
 // be resident at once, one CTA per SM.  Returns W4A4_OK, or -1 when the shape
@@ -522,12 +538,13 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
 }
 
 size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r) {
-  if (M < 0 || !valid_k(K) || (r != 0 && r != 16 && r != 32)) return 0;
+  if (M < 0 || !valid_k(K) || (r != 0 && r != 16 && r != 32) || !valid_lowrank_rows(M, r)) return 0;
   return quant_plan(M, K, r).bytes;
 }
 
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
-  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || (r != 0 && r != 16 && r != 32)) return 0;
+  if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || (r != 0 && r != 16 && r != 32) || !valid_lowrank_rows(M, r))
+    return 0;
   size_t b = quant_plan(M, K, r).bytes;
   b += round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));  // Xq
   b += round256(nvfp4_sf_bytes(M, K));                                  // Xsf
@@ -541,6 +558,7 @@ static int quantize_act_impl(const void* X, int64_t M, int64_t K, int64_t ldx, c
                              size_t workspace_bytes, void* stream, const float* amax_in) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
+  if (!valid_lowrank_rows(M, r)) return W4A4_ERR_SHAPE;
   if (M == 0) return W4A4_OK;  // empty problem: nothing to check further, nothing enqueued
   if (!X || !Xq || !Xsf || !t_x) return W4A4_ERR_NULL;
   if (r > 0 && (!L1t || !t_w || !U)) return W4A4_ERR_NULL;
@@ -644,6 +662,7 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* W
                 int epilogue, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
   if (M < 0 || N <= 0 || N % 8 != 0 || !valid_k(K) || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
+  if (!valid_lowrank_rows(M, r)) return W4A4_ERR_SHAPE;
   if (epilogue != W4A4_EPI_NONE && epilogue != W4A4_EPI_GELU_TANH) return W4A4_ERR_ARG;
   if (M == 0) return W4A4_OK;  // empty problem
   if (!X || !Wq || !Wsf || !t_w || !Y) return W4A4_ERR_NULL;
@@ -681,51 +700,61 @@ int nvfp4_sf_to_rowmajor(const uint8_t* sf_atoms, int64_t rows, int64_t K, uint8
   return W4A4_OK;
 }
 
-int w4a4_device_status(int* status, int reset) {
-  if (!status) return W4A4_ERR_NULL;
-  if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
-  int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
-  *status = v;
-  if (reset) {
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
-  }
-  return W4A4_OK;
-}
 
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
 // Allocation-free activation quantisation.  Its scratch is this file-scope
 // device array; host code cannot use the symbol as a device address, so the
-// address is looked up once per device with cudaGetSymbolAddress.
+// address is looked up with cudaGetSymbolAddress, with the device current.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A4_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void* g_noalloc_ptr[w4a4::kMaxDevices] = {};
+// Per device: the address of the array whose zeroing has been enqueued
+// (nullptr: not yet, or cleared again by w4a4_device_status with reset).
+void* g_noalloc_zeroed[w4a4::kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of g_noalloc_scratch on the current device, or nullptr on
-// failure.  The first call per device also zeroes the array on ``stream``
-// (its counters must start at zero; the kernels leave them zero).
-void* noalloc_scratch(cudaStream_t stream) {
-  int dev = 0;
+int current_device_index() {
+  int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= w4a4::kMaxDevices) {
+    cudaGetLastError();
+    return -1;
+  }
+  return dev;
+}
+
+// Device address of g_noalloc_scratch on the current device, or nullptr on
+// failure.  The address is looked up on every call (a new context on the
+// device loads the module again, possibly elsewhere); the first call for an
+// address zeroes the array on ``stream`` (its counters must start at zero,
+// and the kernels leave them zero).
+void* noalloc_scratch(cudaStream_t stream) {
+  const int dev = current_device_index();
+  if (dev < 0) return nullptr;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
     cudaGetLastError();
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess ||
-        cudaMemsetAsync(ptr, 0, W4A4_NOALLOC_SCRATCH_BYTES, stream) != cudaSuccess) {
+  if (g_noalloc_zeroed[dev] != ptr) {
+    if (cudaMemsetAsync(ptr, 0, W4A4_NOALLOC_SCRATCH_BYTES, stream) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
-    g_noalloc_ptr[dev] = ptr;
+    g_noalloc_zeroed[dev] = ptr;
   }
-  return g_noalloc_ptr[dev];
+  return ptr;
+}
+
+// After a device error: the next no-alloc call on the current device zeroes
+// the array again before it runs.
+void noalloc_mark_dirty() {
+  const int dev = current_device_index();
+  if (dev < 0) return;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  g_noalloc_zeroed[dev] = nullptr;
 }
 }  // namespace
 
@@ -736,6 +765,7 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
                                void* stream) {
   if (M < 0 || !valid_k(K) || ldx < K || ldx % 8 != 0 || M > (int64_t(1) << 30)) return W4A4_ERR_SHAPE;
   if (r != 0 && r != 16 && r != 32) return W4A4_ERR_SHAPE;
+  if (!valid_lowrank_rows(M, r)) return W4A4_ERR_SHAPE;
   if (M == 0) return W4A4_OK;  // empty problem
   const size_t need = nvfp4_quant_workspace_bytes(M, K, r);
   if (need > W4A4_NOALLOC_SCRATCH_BYTES) return W4A4_ERR_SCRATCH_LIMIT;
@@ -748,6 +778,35 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
   if (scratch == nullptr) return W4A4_ERR_CUDA;
   return nvfp4_quantize_act(X, M, K, ldx, inv_s, L1t, r, t_w, Xq, Xsf, t_x, U, scratch,
                             W4A4_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int w4a4_device_status(int* status, int reset) {
+  if (!status) return W4A4_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+  *status = v;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return W4A4_ERR_CUDA; }
+    noalloc_mark_dirty();
+  }
+  return W4A4_OK;
+}
+
+int w4a4_set_wait_bound(int64_t cycles) {
+  if (cycles <= 0) cycles = kDefaultWaitBoundCycles;
+  if (cycles < 1000000) return W4A4_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  const int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  const long long v = cycles;
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyToSymbol(c_wait_bound_cycles, &v, sizeof(v)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  return W4A4_OK;
 }
 
 const char* w4a4_status_string(int status) {

@@ -47,16 +47,18 @@
  *     the legacy default stream).  Scalars (t_x, t_w) stay in device memory.
  *   - Host-detectable problems return an error before anything is enqueued.
  *   - Pointers must be 16-byte aligned; ldx/ldr/ldy are in elements.
- *   - Constraints: K % 256 == 0, K >= 256; N % 8 == 0; r in {0, 16, 32}
+ *   - Constraints: K % 64 == 0, K >= 64 (one FP4 MMA K-step of four 16-element
+ *     scale blocks); N % 8 == 0; r in {0, 16, 32}
  *     (rank 16 is the pages' choice for the low-rank branch, "SVDQuant
  *     Guide ...", "The Solution ..." and "Empirical Efficiency Benchmark");
  *     M >= 0, rows need not be a multiple of 128.  An empty problem (M == 0;
  *     N == 0 for nvfp4_pack_weight; rows == 0 for nvfp4_sf_to_rowmajor) with
  *     valid sizes returns W4A4_OK at once: pointers may then be NULL,
  *     nothing is checked further and nothing is enqueued.
- *   - A device-side pipeline wait that exceeds its bound (about two seconds)
- *     records W4A4_ERR_DEVICE_TIMEOUT in a sticky status word, drains its own
- *     copies and returns; read it with w4a4_device_status() after a sync.
+ *   - A device-side pipeline wait that exceeds its bound (about two seconds,
+ *     see w4a4_set_wait_bound) records W4A4_ERR_DEVICE_TIMEOUT in a sticky
+ *     status word, drains its own copies and returns; read it with
+ *     w4a4_device_status().
  *   - The current CUDA device must be compute capability 10.x (B200 / sm_100a);
  *     there is no fallback.
  */
@@ -92,17 +94,34 @@ enum { W4A4_SRC_BF16 = 0, W4A4_SRC_F32 = 1 };
 size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
 
 /* Workspace bytes needed by nvfp4_quantize_act / nvfp4_pack_weight for an
- * [M, K] input with rank r (amax partial maxima, low-rank partial sums and
- * per-row-block counters).  Returns 0 for invalid sizes.
+ * [M, K] input with rank r (amax partial maxima, the grid-barrier words of the
+ * single-pass quantiser, per-row-block counters and low-rank partial sums).
+ * Returns 0 for invalid sizes.
  *
  * Workspace contract (every entry point that takes a workspace): zero the
  * whole workspace once before its first use (cudaMemset, torch.zeros).  The
  * synchronisation words in it stay valid from call to call (counters are
  * cleared by the call that used them; the single-pass grid barrier keeps a
  * launch generation that every call advances), so no clearing is needed
- * between calls, whatever their sizes.  After a call reports a device error
- * (w4a4_device_status), zero the workspace again.  Calls that overlap on the
- * GPU must not share a workspace. */
+ * between calls, whatever their sizes: the layout below is the same for every
+ * M, K and r, only the length of the last part grows with M.  After a call
+ * reports a device error (w4a4_device_status), zero the workspace again: a
+ * wait that gave up leaves its counters where they stood.  Calls that overlap
+ * on the GPU must not share a workspace.
+ *
+ * Layout (byte offsets from the workspace base):
+ *   0                        amax partial maxima of the two-pass path (fp32 x 1024)
+ *   W4A4_WS_BARRIER_OFFSET   grid barrier: launch generation, arrival counters
+ *                            and tensor-maximum words (160 u32, 128-byte lines)
+ *   W4A4_WS_TICKETS_OFFSET   one u32 counter per 128-row block (row block b at
+ *                            byte W4A4_WS_TICKETS_OFFSET + 4 b), zero at rest
+ *   W4A4_WS_UPART_OFFSET     fp32 low-rank partial sums (r > 0 only)
+ * With a low-rank branch (r > 0) M is at most W4A4_MAX_LOWRANK_ROWS, the
+ * number of rows the counters cover. */
+#define W4A4_WS_BARRIER_OFFSET ((size_t)4096)
+#define W4A4_WS_TICKETS_OFFSET ((size_t)5120)
+#define W4A4_MAX_LOWRANK_ROWS ((int64_t)1 << 22)
+#define W4A4_WS_UPART_OFFSET (W4A4_WS_TICKETS_OFFSET + (size_t)4 * (size_t)(W4A4_MAX_LOWRANK_ROWS / 128))
 size_t nvfp4_quant_workspace_bytes(int64_t M, int64_t K, int r);
 
 /* Workspace bytes needed by w4a4_linear: the quantisation workspace plus the
@@ -242,15 +261,18 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K,
  *   W4A4_NOALLOC_SCRATCH_BYTES are rejected with W4A4_ERR_SCRATCH_LIMIT
  *   before anything is enqueued (with r = 32 this admits roughly M up to
  *   100k tokens).
- * - The first call on a device looks up the device address of the array
- *   (cudaGetSymbolAddress, with that device current), caches it and zeroes
- *   the array on that call's stream; make that first call before any stream
- *   capture.
+ * - Every call looks up the device address of the array on the current
+ *   device (cudaGetSymbolAddress, with that device current); the first call
+ *   for that address zeroes the array on the call's stream, so make the first
+ *   call on a device before any stream capture.
  * - All calls share the one array, which keeps the last call's contents.  The
  *   kernels rewrite every scratch value they read and leave the counters zero
- *   when they end, so no clearing is needed between calls, but calls that
- *   overlap on the GPU (for example on two streams without ordering between
- *   them) race on the array and give wrong results.
+ *   when they end, so no clearing is needed between calls of any sizes (the
+ *   scratch layout does not depend on them; see nvfp4_quant_workspace_bytes),
+ *   but calls that overlap on the GPU (for example on two streams without
+ *   ordering between them) race on the array and give wrong results.
+ * - After a call reports a device error, w4a4_device_status(&st, 1) makes the
+ *   next call on that device zero the array again before it runs.
  */
 #define W4A4_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
@@ -258,9 +280,23 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
                                uint8_t* Xq, uint8_t* Xsf, float* t_x, void* U, void* stream);
 
 /* Copies the sticky device status word of the current device into *status
- * (W4A4_OK, W4A4_ERR_DEVICE_TIMEOUT or W4A4_ERR_DEVICE_LAYOUT) and clears it if reset != 0.  This call
- * synchronises the device.  Returns W4A4_OK or W4A4_ERR_CUDA. */
+ * (W4A4_OK, W4A4_ERR_DEVICE_TIMEOUT or W4A4_ERR_DEVICE_LAYOUT) and clears it
+ * if reset != 0; a reset also makes the next nvfp4_quantize_act_noalloc call
+ * on this device zero its built-in scratch first (caller-owned workspaces the
+ * caller zeroes itself).  This call synchronises the device.  Returns W4A4_OK
+ * or W4A4_ERR_CUDA. */
 int w4a4_device_status(int* status, int reset);
+
+/* Sets how long a device-side wait (pipeline barrier, grid barrier, counter)
+ * spins before it gives up, records W4A4_ERR_DEVICE_TIMEOUT in the sticky
+ * status word, drains its own copies and returns: ``cycles`` SM clock cycles
+ * (at least 1e6), or the default 4e9 (about two seconds at 1.9 GHz) when
+ * cycles <= 0.  Applies to kernels launched on the current device after the
+ * call; synchronises the device.  A short bound lets a caller detect a stuck
+ * pipeline quickly; it must stay well above the longest legitimate wait (a
+ * full-size TMA stage lands within microseconds).  W4A4_ERR_ARG for
+ * 0 < cycles < 1e6. */
+int w4a4_set_wait_bound(int64_t cycles);
 
 /*
  * nvfp4_sf_to_rowmajor -- a layout helper (for checking and debugging): the

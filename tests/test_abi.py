@@ -65,7 +65,7 @@ def test_host_validation_before_any_launch(so):
     big = 1 << 30
     q = w.lib().nvfp4_quantize_act
     assert q(None, 128, 512, 512, None, None, 0, None, P, P, P, None, P, big, None) == -1     # NULL X
-    assert q(P, 128, 500, 512, None, None, 0, None, P, P, P, None, P, big, None) == -2        # K % 256
+    assert q(P, 128, 500, 512, None, None, 0, None, P, P, P, None, P, big, None) == -2        # K % 64
     assert q(P, 128, 512, 500, None, None, 0, None, P, P, P, None, P, big, None) == -2        # ldx < K
     assert q(P, 128, 512, 512, None, None, 24, None, P, P, P, None, P, big, None) == -2       # rank
     assert q(P, 128, 512, 512, None, None, 16, None, P, P, P, None, P, big, None) == -1       # rank 16, no L1t
@@ -78,7 +78,7 @@ def test_host_validation_before_any_launch(so):
     assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 120, None) == -2     # ldy < N
     assert g(P, P, P, None, 128, 128, 512, P, P, P, None, 32, None, 0, P, 128, None) == -1    # no U/L2t
     h = w.lib().nvfp4_sf_to_rowmajor
-    assert h(P, 128, 500, P, None) == -2                                                      # K % 256
+    assert h(P, 128, 500, P, None) == -2                                                      # K % 64
     assert h(None, 128, 512, P, None) == -1                                                   # NULL
     assert h(P, 128, 512, P + 4, None) == -3                                                  # alignment
     pw = w.lib().nvfp4_pack_weight
@@ -94,7 +94,7 @@ def test_host_validation_linear_and_amax_entries(so):
     lin = so.w4a4_linear
     #        X  M    N    K    Wq Wsf t_w inv_s L1t L2t r   bias  epi Y  ws  ws_bytes stream
     assert lin(P, 128, 100, 512, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -2   # N % 8
-    assert lin(P, 128, 128, 500, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -2   # K % 256
+    assert lin(P, 128, 128, 500, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -2   # K % 64
     assert lin(P, 128, 128, 512, P, P, P, None, P, P, 24, None, 0, P, P, big, None) == -2   # rank
     assert lin(P, 128, 128, 512, P, P, P, None, P, P, 32, None, 7, P, P, big, None) == -8   # epilogue
     assert lin(None, 128, 128, 512, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -1  # NULL X
@@ -105,7 +105,7 @@ def test_host_validation_linear_and_amax_entries(so):
     #        X  M    K    ldx inv_s L1t r  t_w  amax   Xq Xsf t_x U     ws  ws_bytes stream
     assert qa(P, 128, 512, 512, None, None, 0, None, None, P, P, P, None, P, big, None) == -1  # no amax
     assert qa(P, 128, 512, 512, None, None, 0, None, P + 2, P, P, P, None, P, big, None) == -3  # amax align
-    assert qa(P, 128, 500, 512, None, None, 0, None, P, P, P, P, None, P, big, None) == -2      # K % 256
+    assert qa(P, 128, 500, 512, None, None, 0, None, P, P, P, P, None, P, big, None) == -2      # K % 64
     gn = so.w4a4_gemm_next_amax
     #       Xq Xsf t_x U     M    N    K    Wq Wsf t_w L2t  r  bias  epi Y  ldy  inv_s  amax   stream
     assert gn(P, P, P, None, 128, 128, 512, P, P, P, None, 0, None, 0, P, 128, None, None, None) == -1
@@ -141,3 +141,51 @@ def test_no_gpu_reports_arch_error(so):
     P = 1 << 20
     st = so.nvfp4_quantize_act(P, 128, 512, 512, None, None, 0, None, P, P, P, None, P, 1 << 30, None)
     assert st == -4
+
+
+def _header_define(name):
+    src = open(HEADER).read()
+    m = re.search(r"#define " + name + r" \((.*)\)\s*$", src, flags=re.M)
+    assert m, name
+    return m.group(1)
+
+
+def test_k_multiple_of_64_is_accepted(so):
+    """One FP4 MMA K-step (64 elements, four scale blocks) is the unit: K =
+    3136 = 49 x 64 passes every size check (and reaches the device check)."""
+    assert so.nvfp4_quant_workspace_bytes(4608, 3136, 32) > 0
+    assert so.nvfp4_quant_workspace_bytes(4608, 64, 0) > 0
+    assert so.nvfp4_quant_workspace_bytes(4608, 3100, 32) == 0
+    assert so.w4a4_workspace_bytes(4608, 9216, 3136, 32) > 0
+    assert so.nvfp4_sf_bytes(128, 3136) == 128 * 196
+    if not __import__("torch").cuda.is_available():
+        P = 1 << 20
+        st = so.nvfp4_quantize_act(P, 128, 3136, 3136, None, None, 0, None, P, P, P, None, P, 1 << 30, None)
+        assert st == -4
+
+
+def test_workspace_layout_does_not_depend_on_the_sizes(so):
+    """The synchronisation words sit at fixed offsets (documented in the
+    header); only the low-rank partial sums at the end grow with M."""
+    bar = int(_header_define("W4A4_WS_BARRIER_OFFSET").split(")")[-1])
+    tick = int(_header_define("W4A4_WS_TICKETS_OFFSET").split(")")[-1])
+    assert (bar, tick) == (4096, 5120)
+    max_rows = 1 << 22
+    upart = tick + 4 * (max_rows // 128)
+    for M, K in [(1, 64), (128, 3072), (4608, 3072), (9216, 3072), (18432, 12288), (16896, 24576)]:
+        b0 = so.nvfp4_quant_workspace_bytes(M, K, 0)
+        b32 = so.nvfp4_quant_workspace_bytes(M, K, 32)
+        assert b0 == upart, (M, K)
+        assert b32 > upart and (b32 - upart) % (128 * 32 * 4) == 0, (M, K)
+    # with a low-rank branch the counters cover at most 2^22 rows
+    assert so.nvfp4_quant_workspace_bytes(max_rows, 64, 32) > 0
+    assert so.nvfp4_quant_workspace_bytes(max_rows + 1, 64, 32) == 0
+    assert so.nvfp4_quant_workspace_bytes(max_rows + 1, 64, 0) > 0
+    P = 1 << 20
+    assert so.nvfp4_quantize_act(P, max_rows + 1, 64, 64, None, P, 32, P, P, P, P, P, P, 1 << 40, None) == -2
+
+
+def test_wait_bound_argument_check(so):
+    assert so.w4a4_set_wait_bound(5) == -8
+    if not __import__("torch").cuda.is_available():
+        assert so.w4a4_set_wait_bound(0) == -4
