@@ -1,17 +1,23 @@
 #!/usr/bin/env python
 """Benchmark of the W4A4 NVFP4 linear hot path on B200.
 
-One step = one pass of the whole hot path over one batch: tensor amax, fused
-smooth/quantise/pack + low-rank down-projection, and the block-scaled FP4 GEMM
-with the low-rank up-projection, bias and bf16 cast, on the FLUX-1024px QKV
-projection (M = 4608 tokens = 4096 image + 512 text, K = 3072, N = 9216,
-rank 32, bf16 bias).  Inputs are synthetic (seeded), shaped like that workload.
+One step = one pass of the whole hot path over one batch, on the 2048px
+large-hidden DiT block (the largest configuration that fits one GPU): for
+each of its two linears -- the fused QKV + SwiGLU-up projection 6144 -> 55296
+and the output projection 24576 -> 6144, M = 16896 tokens (16384 image +
+512 text), rank 32 -- the tensor amax, the fused smooth/quantise/pack +
+low-rank down-projection, and the block-scaled FP4 GEMM with the low-rank
+up-projection and the bf16 cast.  Inputs are synthetic and seeded (per-channel
+lognormal(0, 1.5) activation magnitudes, N(0, 0.02) weights), drawn on the GPU.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload block2048|qkv1024] [--table]
 
 Prints one JSON line.  Under torchrun (N > 1) every rank runs an independent
 replica on its own GPU (the path has no cross-GPU exchange); rank 0 prints.
 ``--impl reference`` times the plain CPU oracle on the host cores instead.
+``--workload qkv1024`` runs the FLUX-1024px QKV projection instead (M = 4608,
+3072 -> 9216); ``--table`` times every configuration's layers.
 """
 from __future__ import annotations
 
@@ -30,21 +36,57 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = {"workload": "FLUX-1024px QKV projection", "M": 4608, "K": 3072, "N": 9216, "r": 32,
-            "bias": True, "activation": "N(0,1) with 1% Student-t(2)x50 channels", "weight": "N(0,0.02)"}
 METRIC = "W4A4 linear TFLOPS (act-quant+FP4 GEMM+low-rank)"
-L2_SETS = 3          # rotating buffer sets, each ~140 MB, so every step starts L2-cold
 MID_EVERY = 10       # steps between per-kernel timing events inside the timed region
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# name -> (description, M, [(layer, K, N)], activation recipe, bias, seed base, L2 sets)
+WORKLOADS = {
+    "block2048": {
+        "workload": "2048px large-hidden DiT block: fused QKV+SwiGLU-up and output linears",
+        "M": 16896, "linears": [("qkv_swiglu_up", 6144, 55296), ("out", 24576, 6144)], "r": 32,
+        "act": "lognormal", "activation": "N(0,1) x per-channel lognormal(0,1.5) magnitudes",
+        "weight": "N(0,0.02)", "bias": False, "seed": 1004, "l2_sets": 1,
+        "l2": "no rotation needed: X2 830 MB and Y1 1.87 GB per step exceed the 126 MB L2, so every kernel "
+              "starts on operands another kernel has evicted"},
+    "qkv1024": {
+        "workload": "FLUX-1024px QKV projection",
+        "M": 4608, "linears": [("qkv", 3072, 9216)], "r": 32,
+        "act": "student_t", "activation": "N(0,1) with 1% Student-t(2)x50 channels",
+        "weight": "N(0,0.02)", "bias": True, "seed": 1002, "l2_sets": 3,
+        "l2": "3 rotating input/weight/output sets of ~140 MB each (> 126 MB L2)"},
+}
+DEFAULT_WORKLOAD = "block2048"
+
+
+def workload_config(name):
+    w = WORKLOADS[name]
+    return {"workload": w["workload"], "M": w["M"],
+            "linears": [{"layer": n, "K": k, "N": nn} for n, k, nn in w["linears"]], "r": w["r"],
+            "bias": w["bias"], "activation": w["activation"], "weight": w["weight"]}
+
+
+WORKLOAD = workload_config(DEFAULT_WORKLOAD)
+
 
 def flops_per_step(M, K, N, r):
+    """Algorithmic work of one linear: the FP4 product and both low-rank projections."""
     return 2.0 * M * N * K + 2.0 * M * r * (K + N)
 
 
 def gemm_flops(M, K, N, r):
-    return 2.0 * M * N * K + 2.0 * M * N * (2 * r)  # main GEMM + the hi/lo low-rank pass
+    """Algorithmic work of the GEMM kernel: the FP4 product and the low-rank up-projection."""
+    return 2.0 * M * N * K + 2.0 * M * r * N
+
+
+def quant_bytes(M, K, r):
+    """Algorithmic bytes of one activation quantisation: the tensor amax reads X
+    once (2MK), the quantise pass reads it again and writes the codes (MK/2),
+    the scale bytes (MK/16) and U (4Mr), and reads inv_s (4K) and L1t (2Kr)."""
+    a0 = 2 * M * K
+    a = 2 * M * K + M * K // 2 + M * K // 16 + 4 * M * r + 4 * K + 2 * K * r
+    return a0, a
 
 
 def load_peaks():
@@ -59,6 +101,7 @@ def load_peaks():
 GEMM_SOURCES = ["bit_diffusion_transformer_nvfp4_b200/csrc/gemm.cuh",
                 "bit_diffusion_transformer_nvfp4_b200/csrc/gemm2.cuh",
                 "bit_diffusion_transformer_nvfp4_b200/csrc/sm100.cuh"]
+GEMM_SUMMARY = {"block2048": "gemm_block2048_up_ncu.md", "qkv1024": "gemm_flux1024_qkv_ncu.md"}
 
 
 def source_hash(paths):
@@ -144,34 +187,71 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
-def build_inputs(torch, w4, prep, dev):
-    from synth import config_cases, bf16_bits
-    case = config_cases(2)[0]
-    M, K, N, r = case.M, case.K, case.N, case.r
+def device_linear_inputs(torch, wl, K, N, seed, dev):
+    """One linear's seeded synthetic inputs, drawn on the GPU with the
+    workload's recipe: activation X [M, K] and a calibration draw [512, K]
+    sharing its outlier structure, bf16 weight [N, K] ~ N(0, 0.02), bf16 bias
+    ~ N(0, 0.01) or none."""
+    M = wl["M"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
 
-    def dev_bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(bf16_bits(a).view(np.int16))).to(dev).view(torch.bfloat16)
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32)
 
-    W = dev_bf16(case.w)
-    Xc = dev_bf16(case.x_cal)
-    bias = dev_bf16(case.bias)
-    packed = prep.svdquant_prepare(W, Xc, r=r, bias=bias)
-    del W, Xc
-    x_host = np.ascontiguousarray(bf16_bits(case.x).view(np.int16))
-    sets = []
-    for i in range(L2_SETS):
-        X = torch.from_numpy(x_host).to(dev).view(torch.bfloat16)
-        w = w4.PackedWeight(packed.Wq.clone(), packed.Wsf.clone(), packed.t_w.clone(), N, K,
-                            packed.inv_s.clone(), packed.L1t.clone(), packed.L2t.clone(), packed.bias.clone())
-        qa = w4.QuantizedActivation(
+    if wl["act"] == "lognormal":
+        mags = torch.exp(1.5 * randn(K))
+        X = (randn(M, K) * mags).to(torch.bfloat16)
+        Xc = (randn(512, K) * mags).to(torch.bfloat16)
+    else:  # 1% of the channels replaced by 50 x Student-t(2) = 50 Z / sqrt(E), E ~ Exp(1)
+        ch = torch.randperm(K, generator=g, device=dev)[:round(0.01 * K)]
+
+        def draw(m):
+            x = randn(m, K)
+            e = -torch.log(torch.rand(m, len(ch), generator=g, device=dev).clamp_min(1e-30))
+            x[:, ch] = 50.0 * randn(m, len(ch)) / torch.sqrt(e)
+            return x.to(torch.bfloat16)
+        X, Xc = draw(M), draw(512)
+    W = (0.02 * randn(N, K)).to(torch.bfloat16)
+    bias = (0.01 * randn(N)).to(torch.bfloat16) if wl["bias"] else None
+    return X, Xc, W, bias
+
+
+class Layer:
+    """Device buffers of one linear of the step."""
+
+    def __init__(self, torch, w4, name, M, K, N, r, X, w, dev):
+        self.name, self.M, self.K, self.N, self.r = name, M, K, N, r
+        self.X, self.w = X, w
+        self.qa = w4.QuantizedActivation(
             torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
             torch.empty(w4.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev),
             torch.empty(1, dtype=torch.float32, device=dev),
             torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev), M, K, r)
-        ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
-        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        sets.append((X, w, qa, ws, Y))
-    return case, x_host, sets
+        self.ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
+        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+
+def build_layers(torch, w4, prep, wl, dev):
+    """Every linear of the workload (``l2_sets`` copies: rotating buffer sets
+    for workloads that would otherwise sit in L2), weights prepared once."""
+    sets = []
+    packed = []
+    for i, (name, K, N) in enumerate(wl["linears"]):
+        X, Xc, W, bias = device_linear_inputs(torch, wl, K, N, wl["seed"] + 100 * i, dev)
+        pk = prep.svdquant_prepare(W, Xc, r=wl["r"], bias=bias)
+        del W, Xc
+        packed.append((name, K, N, X, pk))
+    for s in range(wl["l2_sets"]):
+        layers = []
+        for name, K, N, X, pk in packed:
+            if s > 0:
+                X = X.clone()
+                pk = w4.PackedWeight(pk.Wq.clone(), pk.Wsf.clone(), pk.t_w.clone(), N, K, pk.inv_s.clone(),
+                                     pk.L1t.clone(), pk.L2t.clone(), None if pk.bias is None else pk.bias.clone())
+            layers.append(Layer(torch, w4, name, wl["M"], K, N, wl["r"], X, pk, dev))
+        sets.append(layers)
+    return sets
 
 
 def max_over_ranks(values, world):
@@ -192,6 +272,21 @@ def whole_job_tflops(world, flops_per_rank_step, steps, total_ms):
     return world * flops_per_rank_step * steps / (total_ms * 1e-3) / 1e12
 
 
+def count_library_launches(torch, fn):
+    """Kernels of this library (names in the ``w4a4`` namespace) that one call
+    of ``fn`` launches, from the CUDA activity trace; None if no trace."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+        n = sum(1 for nm in names if "w4a4::" in nm)
+        return n if n > 0 else None
+    except Exception:
+        return None
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -208,89 +303,111 @@ def run_ours(args):
     from bit_diffusion_transformer_nvfp4_b200 import prep
     w4.lib()
 
-    case, x_host, sets = build_inputs(torch, w4, prep, dev)
-    M, K, N, r = case.M, case.K, case.N, case.r
+    wl = WORKLOADS[args.workload]
+    sets = build_layers(torch, w4, prep, wl, dev)
+    n_sets = len(sets)
     stream = torch.cuda.current_stream()
 
-    def step(i, ev_mid=None):
-        X, w, qa, ws, Y = sets[i % L2_SETS]
-        w4.nvfp4_quantize_act(X, M, K, K, w.inv_s, w.L1t, r, w.t_w, qa.Xq, qa.Xsf, qa.t_x, qa.U, ws, stream)
-        if ev_mid is not None:
-            ev_mid.record(stream)
-        w4.w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, w.Wq, w.Wsf, w.t_w, w.L2t, r, w.bias, 0, Y, N, stream)
+    def quant(L):
+        w = L.w
+        w4.nvfp4_quantize_act(L.X, L.M, L.K, L.K, w.inv_s, w.L1t, L.r, w.t_w, L.qa.Xq, L.qa.Xsf, L.qa.t_x, L.qa.U,
+                              L.ws, stream)
+
+    def gemm(L):
+        w = L.w
+        w4.w4a4_gemm(L.qa.Xq, L.qa.Xsf, L.qa.t_x, L.qa.U, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.L2t, L.r, w.bias, 0,
+                     L.Y, L.N, stream)
+
+    def step(i, evs=None):
+        for j, L in enumerate(sets[i % n_sets]):
+            quant(L)
+            if evs is not None:
+                evs[2 * j + 1].record(stream)
+            gemm(L)
+            if evs is not None:
+                evs[2 * j + 2].record(stream)
 
     def barrier():
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
 
-    sampler = ClockSampler(local)
-    sampler.start()
     for i in range(args.warmup):
         step(i)
     barrier()
+    per_step_launches = None if args.no_profile else count_library_launches(torch, lambda: step(0))
+    barrier()
+    n_lin = len(wl["linears"])
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
     # One event pair brackets the timed steps.  Every MID_EVERY-th step also
-    # records events before the quantiser, between the kernels and after the
+    # records events before the first kernel and after each quantiser and
     # GEMM (the per-kernel durations).  An event between two kernels makes
     # the second wait for the first to finish instead of starting its set-up
     # early (programmatic launch), so the other steps go without them.
     ev_first, ev_last = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampled = list(range(0, args.steps, MID_EVERY))
-    evs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-               torch.cuda.Event(enable_timing=True)) for i in sampled}
+    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_lin + 1)] for i in sampled}
     t_wall0 = time.time()
     ev_first.record(stream)
     for i in range(args.steps):
         if i in evs:
             evs[i][0].record(stream)
-            step(i, evs[i][1])
-            evs[i][2].record(stream)
+            step(i, evs[i])
         else:
             step(i)
     ev_last.record(stream)
     barrier()
     t_wall1 = time.time()
+    clock_rows = sampler.stop()
     total_ms = ev_first.elapsed_time(ev_last)
-    gemm_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in sampled]
-    quant_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in sampled]
+    quant_ms = [statistics.mean(evs[i][2 * j].elapsed_time(evs[i][2 * j + 1]) for i in sampled) for j in range(n_lin)]
+    gemm_ms = [statistics.mean(evs[i][2 * j + 1].elapsed_time(evs[i][2 * j + 2]) for i in sampled)
+               for j in range(n_lin)]
 
     # End to end through the public API with host buffers: every step copies
-    # its X in from pinned host memory, runs w4a4_linear and copies its Y out
-    # to pinned host memory.  Steps are pipelined over three streams (copy in,
-    # compute, copy out) and two device buffer sets, as a serving loop would
-    # run them: one step's copies overlap its neighbours' work, and events keep
-    # the order within a step and the reuse of each buffer set.
-    import torch as _t
-    xh = _t.from_numpy(x_host).view(_t.bfloat16).pin_memory()
-    yh = [_t.empty(M, N, dtype=_t.bfloat16).pin_memory() for _ in range(2)]
-    e2e_steps = max(3, min(args.steps, 50))
-    w0 = sets[0][1]
-    bufs = [(sets[j][0], sets[j][4]) for j in range(2)]
-    lin_ws = w4.new_workspace(w4.w4a4_workspace_bytes(M, N, K, r), dev)
+    # each linear's X in from pinned host memory, runs w4a4_linear on it and
+    # copies its Y out to pinned host memory.  Steps are pipelined over three
+    # streams (copy in, compute, copy out) and two device buffer sets, as a
+    # serving loop would run them: one step's copies overlap its neighbours'
+    # work, and events keep the order within a step and the reuse of each
+    # buffer set.
+    layers0 = sets[0]
+    xh = [L.X.cpu().pin_memory() for L in layers0]
+    yh = [[torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory() for L in layers0] for _ in range(2)]
+    bufs = [[(L.X, L.Y) for L in layers0]]
+    bufs.append([(torch.empty_like(L.X), torch.empty_like(L.Y)) for L in layers0])
+    lin_ws = [w4.new_workspace(w4.w4a4_workspace_bytes(L.M, L.N, L.K, L.r), dev) for L in layers0]
     s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
 
     def e2e_run(n, e_start=None, e_end=None):
         done_c, done_out = [], []
         if e_start is not None:
             e_start.record(s_in)
         for i in range(n):
-            X, Y = bufs[i % 2]
+            b = bufs[i % 2]
             if i >= 2:
-                s_in.wait_event(done_c[i - 2])        # step i-2 no longer reads this X
+                s_in.wait_event(done_c[i - 2])        # step i-2 no longer reads these X
             with torch.cuda.stream(s_in):
-                X.copy_(xh, non_blocking=True)
+                for (X, _), h in zip(b, xh):
+                    X.copy_(h, non_blocking=True)
             ev_in = torch.cuda.Event()
             ev_in.record(s_in)
             s_c.wait_event(ev_in)
             if i >= 2:
-                s_c.wait_event(done_out[i - 2])       # step i-2's Y has been copied out
-            w4.w4a4_linear(X, M, N, K, w0.Wq, w0.Wsf, w0.t_w, w0.inv_s, w0.L1t, w0.L2t, r, w0.bias, 0, Y,
-                           lin_ws, s_c)
+                s_c.wait_event(done_out[i - 2])       # step i-2's Y have been copied out
+            for (X, Y), L, ws in zip(b, layers0, lin_ws):
+                w = L.w
+                w4.w4a4_linear(X, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.inv_s, w.L1t, w.L2t, L.r, w.bias, 0, Y, ws,
+                               s_c)
             ev_c = torch.cuda.Event()
             ev_c.record(s_c)
             s_out.wait_event(ev_c)
             with torch.cuda.stream(s_out):
-                yh[i % 2].copy_(Y, non_blocking=True)
+                for (_, Y), h in zip(b, yh[i % 2]):
+                    h.copy_(Y, non_blocking=True)
             ev_out = torch.cuda.Event()
             ev_out.record(s_out)
             done_c.append(ev_c)
@@ -298,57 +415,79 @@ def run_ours(args):
         if e_end is not None:
             e_end.record(s_out)
 
-    e2e_run(4)
+    e2e_run(2)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_run(e2e_steps, e0, e1)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    clock_rows = sampler.stop()
     status = w4.w4a4_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status}: {w4.w4a4_status_string(status)}")
 
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world)
+    total_ms, e2e_ms, *kern = max_over_ranks([total_ms, e2e_ms, *quant_ms, *gemm_ms], world)
+    quant_ms, gemm_ms = kern[:n_lin], kern[n_lin:]
 
-    fl = flops_per_step(M, K, N, r)
+    M, r = wl["M"], wl["r"]
+    fl = sum(flops_per_step(M, K, N, r) for _, K, N in wl["linears"])
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(world, fl, args.steps, total_ms)
     peaks, peak_kind = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    gemm_avg_ms = statistics.mean(gemm_ms)
-    g_fl = gemm_flops(M, K, N, r)
-    achieved = g_fl / (gemm_avg_ms * 1e-3) / 1e12
-    traffic = ncu_traffic(GEMM_SOURCES, "gemm_flux1024_qkv_ncu.md")
+    fp4_peak_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * FP4_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    rooflines = []
+    for j, (name, K, N) in enumerate(wl["linears"]):
+        g_fl = gemm_flops(M, K, N, r)
+        ach = g_fl / (gemm_ms[j] * 1e-3) / 1e12
+        a0, a = quant_bytes(M, K, r)
+        qach = (a0 + a) / (quant_ms[j] * 1e-3) / 1e9
+        rooflines.append({"kernel": f"gemm2_kernel ({name})", "bound": "tensor", "achieved": round(ach, 2),
+                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(ach / fp4_peak, 4),
+                          "frac_of_sustained": round(ach / fp4_peak_sus, 4), "launch_ms": round(gemm_ms[j], 5),
+                          "algorithmic_flops_per_launch": g_fl})
+        rooflines.append({"kernel": f"activation quantiser ({name}: tensor amax + quantise pass)", "bound": "hbm",
+                          "achieved": round(qach, 1), "peak": hbm, "unit": "GB/s", "frac": round(qach / hbm, 4),
+                          "launch_ms": round(quant_ms[j], 5), "algorithmic_bytes_per_call": a0 + a,
+                          "bytes_basis": "amax pass 2MK + quantise pass 2MK + MK/2 + MK/16 + 4Mr + 4K + 2Kr"})
+    top = max(range(n_lin), key=lambda j: gemm_ms[j])
+    dom = dict(rooflines[2 * top])
+    dom["traffic"] = ncu_traffic(GEMM_SOURCES, GEMM_SUMMARY[args.workload]) if top == 0 else None
+    dom["peak_kind"] = (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16:g} (nominal "
+                        f"FP4/BF16 ratio); frac_of_sustained uses the sustained bf16 figure x {FP4_OVER_BF16:g}")
     clocks = ClockSampler.summarise(clock_rows)
+    if per_step_launches is None:
+        per_step_launches = sum(1 + (2 if 2 * M * K > 64 << 20 else 1) for _, K, _n in wl["linears"])
+        launch_basis = "expected per step (no activity trace)"
+    else:
+        launch_basis = "counted per step from the CUDA activity trace of one step"
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
-        "data": "synthetic",
-        "config": dict(WORKLOAD, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                       l2=f"{L2_SETS} rotating input/weight/output sets of ~140 MB each (> 126 MB L2)"),
+        "data": "synthetic (seeded, drawn on the GPU)",
+        "config": dict(workload_config(args.workload),
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU", l2=wl["l2"]),
         "pct_fp4_peak": round(100.0 * value / (world * fp4_peak), 2),
         "fp4_peak_tflops": round(fp4_peak, 1),
         "fp4_peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOPS x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
-        "roofline": {"kernel": "gemm2_kernel (CTA-pair block-scaled FP4 + low-rank + bias epilogue)", "bound": "tensor",
-                     "achieved": round(achieved, 2), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
-                     "peak_kind": f"{peak_kind} (bf16 burst x4)", "launch_ms": round(gemm_avg_ms, 5),
-                     "algorithmic_flops_per_launch": g_fl},
-        "kernels_ms": {"amax+quant": round(statistics.mean(quant_ms), 5), "gemm": round(gemm_avg_ms, 5),
-                       "sampled_steps": len(gemm_ms)},
+        "roofline": dom,
+        "rooflines": rooflines,
+        "kernels_ms": {**{f"quant_{n}": round(quant_ms[j], 5) for j, (n, _, _) in enumerate(wl["linears"])},
+                       **{f"gemm_{n}": round(gemm_ms[j], 5) for j, (n, _, _) in enumerate(wl["linears"])},
+                       "sampled_steps": len(sampled)},
         "e2e": {"value": round(whole_job_tflops(world, fl, 1, e2e_ms), 2), "unit": "TFLOPS",
-                "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 2),
-                "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear",
+                "h2d_bytes_per_step": int(sum(2 * M * K for _, K, _ in wl["linears"])),
+                "d2h_bytes_per_step": int(sum(2 * M * N for _, _, N in wl["linears"])),
+                "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear", "steps": e2e_steps,
                 "pipelining": "copy-in, compute and copy-out on three streams, two buffer sets"},
-        # per step: the single-pass quantiser and the pair GEMM
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": per_step_launches * args.steps,
+        "gpu_launches_basis": launch_basis,
         "clocks": clocks,
         "wall_s_timed": round(t_wall1 - t_wall0, 3),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(case, args.cpu_rows, args.cpu_cols)
+        out["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows, args.cpu_cols)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -576,8 +715,7 @@ def run_table(args):
     del w_cat
     for B in (1, 2, 4):
         M = 4608 * B
-        acts = [dev_bf16(np.concatenate([trajectory_step_activation(t, 4608, K)[0]] * B, axis=0))
-                for t in range(3)]
+        acts = [dev_bf16(trajectory_step_activation(t, M, K)[0]) for t in range(3)]
         ws1 = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, 32), dev)
         ws2 = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, dn.K, 32), dev)
         qa1 = w4.quantize_act(acts[0], pf.inv_s, pf.L1t, pf.t_w, workspace=ws1)
@@ -629,72 +767,76 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def oracle_prepared(case, cols):
-    """Oracle-side preparation (not timed): smoothing, SVD, and the NVFP4
-    packing of the weight rows of the sampled output channels under the whole
-    residual's tensor scale."""
+def oracle_samples(wl, n_rows, n_cols):
+    """A bounded sample of every linear of the workload, drawn with the same
+    recipe (synth): ``n_rows`` tokens x ``n_cols`` output channels at the
+    layer's full K, with the oracle's preparation done (not timed)."""
     from oracle import nvfp4, prep
-    p = prep.svdquant_prepare(case.w, case.x_cal, case.r, case.alpha)
-    R = p["R"]
-    codes, wsf, tw, _ = nvfp4.quantize(R[cols], amax=np.max(np.abs(R)))
-    return p, nvfp4.pack(codes), wsf, tw
+    from synth import make_linear
+    out = []
+    act = "lognormal" if wl["act"] == "lognormal" else "student_t"
+    for i, (name, K, N) in enumerate(wl["linears"]):
+        c = make_linear(name, n_rows, K, n_cols, r=wl["r"], act=act, bias_std=0.01 if wl["bias"] else 0.0,
+                        seed=wl["seed"] + 100 * i)
+        p = prep.svdquant_prepare(c.w, c.x_cal, c.r, c.alpha)
+        wq, wsf, tw, _ = nvfp4.quantize_activation(p["R"], None)
+        out.append((c, p, wq, wsf, tw))
+    return out
 
 
-def sample_indices(case, rows, cols):
-    g = np.random.Generator(np.random.PCG64(7))
-    return (np.sort(g.choice(case.M, rows, replace=False)), np.sort(g.choice(case.N, cols, replace=False)))
-
-
-def oracle_step(case, prepared, rows, cols):
+def oracle_step(samples):
     from oracle import linear as olinear
-    p, wq, wsf, tw = prepared
-    olinear.w4a4_linear(case.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"][cols],
-                        None if case.bias is None else case.bias[cols], rows=rows)
+    for c, p, wq, wsf, tw in samples:
+        olinear.w4a4_linear(c.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"], c.bias)
 
 
-def cpu_baseline(case, n_rows=1024, n_cols=2048, min_seconds=10.0):
-    """The oracle as it stands on a bounded sample of the workload: the whole
-    activation's tensor scale, then quantisation of ``n_rows`` sampled tokens
-    and Y for them on ``n_cols`` sampled output channels (numpy fp32
-    quantiser, fp64 matmul).  Throughput counts the sample's FLOPs."""
-    rows, cols = sample_indices(case, n_rows, n_cols)
-    prepared = oracle_prepared(case, cols)
+def sample_flops(wl, n_rows, n_cols):
+    return sum(flops_per_step(n_rows, K, n_cols, wl["r"]) for _, K, _ in wl["linears"])
+
+
+def sample_text(wl, n_rows, n_cols):
+    layers = ", ".join(f"{name} K={K}" for name, K, _ in wl["linears"])
+    return (f"{n_rows} of {wl['M']} tokens x {n_cols} output channels of each linear ({layers}), drawn with the "
+            f"workload's recipe; the sample's own tensor scale")
+
+
+def cpu_baseline(wl, n_rows=256, n_cols=1024, min_seconds=10.0):
+    """The oracle as it stands on a bounded sample of the workload (numpy fp32
+    quantiser, fp64 matmul); throughput counts the sample's FLOPs."""
+    samples = oracle_samples(wl, n_rows, n_cols)
     iters = 0
     t0 = time.perf_counter()
     while True:
-        oracle_step(case, prepared, rows, cols)
+        oracle_step(samples)
         iters += 1
         dt = time.perf_counter() - t0
         if dt >= min_seconds:
             break
-    fl = flops_per_step(n_rows, case.K, n_cols, case.r) * iters
+    fl = sample_flops(wl, n_rows, n_cols) * iters
     return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{n_rows} of {case.M} tokens x {n_cols} of {case.N} output channels, K={case.K}, "
-                      f"whole-tensor activation scale; repeated {iters}x in {dt:.1f} s"}
+            "sample": sample_text(wl, n_rows, n_cols) + f"; repeated {iters}x in {dt:.1f} s"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from synth import config_cases
-    case = config_cases(2)[0]
-    rows, cols = sample_indices(case, args.ref_rows, args.ref_cols)
-    prepared = oracle_prepared(case, cols)
+    wl = WORKLOADS[getattr(args, "workload", DEFAULT_WORKLOAD)]
+    samples = oracle_samples(wl, args.ref_rows, args.ref_cols)
     for _ in range(args.warmup):
-        oracle_step(case, prepared, rows, cols)
+        oracle_step(samples)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(case, prepared, rows, cols)
+        oracle_step(samples)
     dt = time.perf_counter() - t0
-    fl = flops_per_step(args.ref_rows, case.K, args.ref_cols, case.r)
+    fl = sample_flops(wl, args.ref_rows, args.ref_cols)
     value = fl * args.steps / dt / 1e12
-    sample = (f"per step: {args.ref_rows} of {case.M} tokens x {args.ref_cols} of {case.N} output channels, "
-              f"K={case.K}, whole-tensor activation scale")
+    sample = "per step: " + sample_text(wl, args.ref_rows, args.ref_cols)
+    name = getattr(args, "workload", DEFAULT_WORKLOAD)
     out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": 0,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": dict(WORKLOAD, parallelism="host CPU"),
+           "config": dict(workload_config(name), parallelism="host CPU"),
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cpu_threads(), "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -704,14 +846,18 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-rows", type=int, default=1024)
-    ap.add_argument("--cpu-cols", type=int, default=2048)
-    ap.add_argument("--ref-rows", type=int, default=256)
-    ap.add_argument("--ref-cols", type=int, default=1024)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--cpu-cols", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--ref-cols", type=int, default=128)
+    ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-profile", action="store_true",
+                    help="skip the activity trace that counts the library's kernel launches (e.g. under ncu)")
     ap.add_argument("--table", action="store_true",
                     help="time every configuration's layers (one JSON line per row) instead of the benchmark step")
     ap.add_argument("--table-reps", type=int, default=20)

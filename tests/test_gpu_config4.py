@@ -1,13 +1,17 @@
-"""GPU parity on the 2048px workload shapes (the largest configuration):
-fused QKV + MLP-up 6144 -> 55296 and the output projection 24576 -> 6144, at
-2112 tokens (a ragged 17th row block) with full K and N.
+"""GPU parity on the 2048px large-hidden block (the largest configuration):
+the fused QKV + SwiGLU-up linear 6144 -> 55296 and the output linear
+24576 -> 6144, at the full 16896 tokens and at 2112 tokens (a ragged 17th row
+block), with full K and N.
 
-The GPU packs the whole residual itself; the sampled weight rows are checked
-bit for bit against the oracle's quantiser (under the whole residual's tensor
-scale), then Y on sampled tokens x sampled output channels against the
-oracle's fp64 result from those same oracle bytes.  The 24576-deep projection
-needs more K slices than can be co-resident, so it also runs the two-pass
-activation quantiser on bf16 input.
+* Weights: the GPU packs the whole residual; sampled rows of its packing are
+  compared with the oracle's bytes under the whole residual's tensor scale.
+* Activations at full size: every code byte and every scale byte of the
+  16896-token activation is compared with the oracle, which quantises the
+  rows in chunks under the whole tensor's amax (rows are independent once the
+  tensor scale is fixed).  Both activations are too large to be co-resident,
+  so they take the two-pass quantiser.
+* Y: sampled tokens x sampled output channels against the oracle's fp64
+  result from those same oracle bytes.
 """
 import numpy as np
 import pytest
@@ -18,6 +22,8 @@ from oracle import nvfp4, prep
 from synth import config_cases, rng
 
 pytestmark = pytest.mark.gpu
+
+CHUNK = 2048  # oracle rows per chunk
 
 
 @pytest.fixture(scope="module")
@@ -30,39 +36,87 @@ def w4():
 
 
 @pytest.fixture(scope="module")
-def cases():
-    return config_cases(4, scale_m=0.125)
+def layers(w4):
+    """Both linears: the full-size case, its oracle preparation and the GPU packing."""
+    import torch
+    out = []
+    for c in config_cases(4):
+        p = prep.svdquant_prepare(c.w, c.x_cal, c.r, c.alpha)
+        pw = w4.pack_weight(to_dev_f32(p["R"]))
+        torch.cuda.synchronize()
+        w = w4.PackedWeight(pw.Wq, pw.Wsf, pw.t_w, c.N, c.K, to_dev_f32(p["inv_s"]), to_dev_bf16(p["L1t"]),
+                            to_dev_bf16(p["L2t"]), to_dev_bf16(c.bias) if c.bias is not None else None)
+        out.append((c, p, w))
+    return out
+
+
+def check_weight_rows(w, p, cols):
+    """Sampled rows of the GPU packing against the oracle; returns the oracle bytes."""
+    oq, osf, ot, _ = nvfp4.quantize(p["R"][cols], amax=np.max(np.abs(p["R"])))
+    owq = nvfp4.pack(oq)
+    assert float(w.t_w.cpu()[0]) == float(ot)
+    np.testing.assert_array_equal(w.Wq.cpu().numpy()[cols], owq)
+    np.testing.assert_array_equal(sf_atoms_to_rowmajor(w.Wsf.cpu().numpy(), w.N, w.K)[cols], osf)
+    return owq, osf, ot
+
+
+def sample(M, N, which, n_rows=96, n_cols=384):
+    g = rng(4000 + which + M)
+    rows = np.sort(g.choice(M, n_rows, replace=False))
+    rows[-1] = M - 1
+    cols = np.sort(g.choice(N, n_cols, replace=False))
+    cols[-1] = N - 1
+    return rows, cols
 
 
 @pytest.mark.parametrize("which", [0, 1])
-def test_config4_sampled(w4, cases, which):
+def test_config4_full_size(w4, layers, which):
     import torch
-    c = cases[which]
-    p = prep.svdquant_prepare(c.w, c.x_cal, c.r, c.alpha)
-    g = rng(4000 + which)
-    rows = np.sort(g.choice(c.M, 96, replace=False))
-    rows[-1] = c.M - 1                           # the ragged last row block
-    cols = np.sort(g.choice(c.N, 384, replace=False))
-    cols[-1] = c.N - 1
+    c, p, w = layers[which]
+    M, K = c.M, c.K
+    assert M == 16896
+    rows, cols = sample(M, c.N, which)
+    owq, osf, ot = check_weight_rows(w, p, cols)
 
-    # the GPU packs the whole residual
-    pw = w4.pack_weight(to_dev_f32(p["R"]))
+    qa = w4.quantize_act(to_dev_bf16(c.x), w.inv_s, w.L1t, w.t_w)
+    Y = w4.gemm(qa, w)
     torch.cuda.synchronize()
-    # oracle bytes of the sampled weight rows under the whole residual's scale
-    oq, osf, ot, _ = nvfp4.quantize(p["R"][cols], amax=np.max(np.abs(p["R"])))
-    owq = nvfp4.pack(oq)
-    assert float(pw.t_w.cpu()[0]) == float(ot)
-    gwq = pw.Wq.cpu().numpy()[cols]
-    gsf = sf_atoms_to_rowmajor(pw.Wsf.cpu().numpy(), c.N, c.K)[cols]
-    np.testing.assert_array_equal(gwq, owq)
-    np.testing.assert_array_equal(gsf, osf)
+    assert w4.w4a4_device_status() == 0
 
-    w = w4.PackedWeight(pw.Wq, pw.Wsf, pw.t_w, c.N, c.K, to_dev_f32(p["inv_s"]), to_dev_bf16(p["L1t"]),
-                        to_dev_bf16(p["L2t"]), to_dev_bf16(c.bias) if c.bias is not None else None)
-    Y = w4.linear(to_dev_bf16(c.x), w)
+    # every activation code and scale byte, in row chunks under the whole tensor's amax
+    amax = np.float32(0.0)
+    for r0 in range(0, M, CHUNK):
+        amax = max(amax, np.float32(np.max(np.abs(nvfp4.smooth(c.x[r0:r0 + CHUNK], p["inv_s"])))))
+    t_x = float(qa.t_x.cpu()[0])
+    assert t_x == float(nvfp4.tensor_scale(amax))
+    gq = qa.Xq.cpu().numpy()
+    gsf = sf_atoms_to_rowmajor(qa.Xsf.cpu().numpy(), M, K)
+    for r0 in range(0, M, CHUNK):
+        codes, sf, t, _ = nvfp4.quantize(nvfp4.smooth(c.x[r0:r0 + CHUNK], p["inv_s"]), amax=amax)
+        assert float(t) == t_x
+        np.testing.assert_array_equal(gq[r0:r0 + CHUNK], nvfp4.pack(codes), err_msg=f"codes, rows from {r0}")
+        np.testing.assert_array_equal(gsf[r0:r0 + CHUNK], sf, err_msg=f"scales, rows from {r0}")
+    del gq, gsf
+
+    y = from_dev_bf16(Y[torch.from_numpy(rows).cuda()])[:, cols]
+    y_ref, _ = olinear.w4a4_linear(c.x, p["inv_s"], owq, osf, ot, p["L1t"], p["L2t"][cols],
+                                   None if c.bias is None else c.bias[cols], rows=rows)
+    check_y(y, y_ref)
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_config4_ragged_rows(w4, layers, which):
+    """2112 tokens (16.5 row blocks) through w4a4_linear, sampled Y."""
+    import torch
+    c, p, w = layers[which]
+    M = 2112
+    x = c.x[:M]
+    rows, cols = sample(M, c.N, which)
+    owq, osf, ot = check_weight_rows(w, p, cols)
+    Y = w4.linear(to_dev_bf16(x), w)
     torch.cuda.synchronize()
     assert w4.w4a4_device_status() == 0
     y = from_dev_bf16(Y)[rows][:, cols]
-    y_ref, _ = olinear.w4a4_linear(c.x, p["inv_s"], owq, osf, ot, p["L1t"], p["L2t"][cols],
-                                   None if c.bias is None else c.bias[cols], rows=rows)
+    y_ref, aux = olinear.w4a4_linear(x, p["inv_s"], owq, osf, ot, p["L1t"], p["L2t"][cols],
+                                     None if c.bias is None else c.bias[cols], rows=rows)
     check_y(y, y_ref)

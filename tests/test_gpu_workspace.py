@@ -2,13 +2,16 @@
 
 The quantiser's per-row-block tickets of the low-rank sums (zero at rest:
 every call clears what it used) and the single-pass grid barrier (a launch
-generation that every call advances, and one tagged slot per CTA) live in
-the caller's workspace.  Here one shared workspace runs the
-single-pass cooperative path, the two-pass path (an activation too large to
-be co-resident) and the quantise-with-given-amax path, in an order that
-changes the grid size and the number of row blocks between calls; every
-result must equal the oracle's bytes (small shapes) or a fresh-workspace
-call's bytes (large shapes), and the device status must stay clean.
+generation that every call advances, with a counter and a maximum word per
+generation parity) live at fixed offsets of the caller's workspace, whatever
+the call's sizes.  Here one shared workspace runs the single-pass
+cooperative path, the two-pass path (an activation too large to be
+co-resident) and the quantise-with-given-amax path, in an order that changes
+the grid size and the number of row blocks between calls, across 64 and 128
+row blocks and back (a layout that moved with M would put one call's
+low-rank partial sums on another call's counters); every result must equal
+the oracle's bytes (small shapes) or a fresh-workspace call's bytes (large
+shapes), and the device status must stay clean.
 """
 import numpy as np
 import pytest
@@ -28,6 +31,12 @@ SEQ = [  # (M, K, r, path)
     (4608, 3072, 32, "measured"),    # single pass again after all of the above
     (4608, 3072, 32, "given"),
     (128, 3072, 32, "measured"),
+    (9216, 3072, 32, "measured"),    # 72 row blocks: two passes
+    (18432, 3072, 32, "measured"),   # 144 row blocks
+    (4608, 3072, 32, "measured"),    # 36 row blocks again: single pass
+    (18432, 3072, 32, "given"),
+    (9216, 3072, 16, "measured"),
+    (300, 512, 32, "measured"),
 ]
 
 
