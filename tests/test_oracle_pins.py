@@ -375,3 +375,41 @@ def test_row_maxabs_ratio_by_hand():
     b = a + np.array([[1.0, 0.0], [0.5, 0.0], [0.0, -1.0]])
     assert linear.row_maxabs_ratio(b, a) == 0.5
     assert linear.row_maxabs_ratio(b[::-1], a[::-1]) == 0.5
+
+
+# ---------------------------------------------------------------- SwiGLU
+
+def test_silu_closed_forms():
+    from oracle import swiglu
+    assert swiglu.silu(np.array([0.0]))[0] == 0.0
+    # sigmoid(ln 3) = 3/4, sigmoid(-ln 3) = 1/4
+    ln3 = np.log(3.0)
+    np.testing.assert_allclose(swiglu.silu(np.array([ln3, -ln3])), [0.75 * ln3, -0.25 * ln3], rtol=1e-15)
+    # silu(x) - silu(-x) = x (sigmoid(x) + sigmoid(-x) = 1), for any x
+    x = np.linspace(-30, 30, 601)
+    np.testing.assert_allclose(swiglu.silu(x) - swiglu.silu(-x), x, rtol=1e-14, atol=1e-14)
+    # limits: x for large x, 0 (from below) for very negative x, no overflow warning
+    assert swiglu.silu(np.array([800.0]))[0] == 800.0
+    v = swiglu.silu(np.array([-800.0]))[0]
+    assert v == 0.0 and np.signbit(v)
+
+
+def test_silu_against_library():
+    torch = pytest.importorskip("torch")
+    from oracle import swiglu
+    x = np.linspace(-20, 20, 2001)
+    ref = torch.nn.functional.silu(torch.tensor(x, dtype=torch.float64)).numpy()
+    np.testing.assert_allclose(swiglu.silu(x), ref, rtol=1e-15, atol=1e-300)
+
+
+def test_swiglu_split_by_hand():
+    from oracle import swiglu
+    # plain 2 columns, then gate (2) and up (2)
+    y = np.array([[1.0, 2.0, 0.0, np.log(3.0), 5.0, 4.0]])
+    plain, h = swiglu.split_fused(y, 2, 2)
+    np.testing.assert_array_equal(plain, [[1.0, 2.0]])
+    # silu(0) * 5 = 0; silu(ln 3) * 4 = 0.75 ln 3 * 4 = 3 ln 3
+    np.testing.assert_allclose(h, [[0.0, 3.0 * np.log(3.0)]], rtol=1e-15)
+    # gate and up are not interchangeable
+    _, h2 = swiglu.split_fused(y[:, [0, 1, 4, 5, 2, 3]], 2, 2)
+    assert not np.allclose(h, h2)
