@@ -46,13 +46,15 @@ WORKLOADS = {
     "block2048": {
         "workload": "2048px large-hidden DiT block: fused QKV+SwiGLU-up and output linears",
         "M": 16896, "linears": [("qkv_swiglu_up", 6144, 55296), ("out", 24576, 6144)], "r": 32,
+        # the fused projection: 3 x 6144 plain QKV features, then 18432 SwiGLU gate/up pairs
+        "swiglu": {"qkv_swiglu_up": 18432},
         "act": "lognormal", "activation": "N(0,1) x per-channel lognormal(0,1.5) magnitudes",
         "weight": "N(0,0.02)", "bias": False, "seed": 1004, "l2_sets": 1,
         "l2": "no rotation needed: X2 830 MB and Y1 1.87 GB per step exceed the 126 MB L2, so every kernel "
               "starts on operands another kernel has evicted"},
     "qkv1024": {
         "workload": "FLUX-1024px QKV projection",
-        "M": 4608, "linears": [("qkv", 3072, 9216)], "r": 32,
+        "M": 4608, "linears": [("qkv", 3072, 9216)], "r": 32, "swiglu": {},
         "act": "student_t", "activation": "N(0,1) with 1% Student-t(2)x50 channels",
         "weight": "N(0,0.02)", "bias": True, "seed": 1002, "l2_sets": 3,
         "l2": "3 rotating input/weight/output sets of ~140 MB each (> 126 MB L2)"},
@@ -62,8 +64,14 @@ DEFAULT_WORKLOAD = "block2048"
 
 def workload_config(name):
     w = WORKLOADS[name]
+
+    def lin(n, k, nn):
+        d = {"layer": n, "K": k, "N": nn}
+        if n in w["swiglu"]:
+            d["epilogue"] = f"SwiGLU: {w['swiglu'][n]} plain outputs, {(nn - w['swiglu'][n]) // 2} silu(gate)*up outputs"
+        return d
     return {"workload": w["workload"], "M": w["M"],
-            "linears": [{"layer": n, "K": k, "N": nn} for n, k, nn in w["linears"]], "r": w["r"],
+            "linears": [lin(n, k, nn) for n, k, nn in w["linears"]], "r": w["r"],
             "bias": w["bias"], "activation": w["activation"], "weight": w["weight"]}
 
 
@@ -220,8 +228,9 @@ def device_linear_inputs(torch, wl, K, N, seed, dev):
 class Layer:
     """Device buffers of one linear of the step."""
 
-    def __init__(self, torch, w4, name, M, K, N, r, X, w, dev):
+    def __init__(self, torch, w4, name, M, K, N, r, X, w, dev, n_plain=None):
         self.name, self.M, self.K, self.N, self.r = name, M, K, N, r
+        self.n_plain = N if n_plain is None else n_plain   # < N: SwiGLU pairs after the plain rows
         self.X, self.w = X, w
         self.qa = w4.QuantizedActivation(
             torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
@@ -229,7 +238,11 @@ class Layer:
             torch.empty(1, dtype=torch.float32, device=dev),
             torch.empty(M, 2 * r, dtype=torch.bfloat16, device=dev), M, K, r)
         self.ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
-        self.Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.Y = torch.empty(M, self.n_plain, dtype=torch.bfloat16, device=dev)
+        self.H = torch.empty(M, (N - self.n_plain) // 2, dtype=torch.bfloat16, device=dev) if self.n_plain < N else None
+
+    def outputs(self):
+        return [self.Y] if self.H is None else [self.Y, self.H]
 
 
 def build_layers(torch, w4, prep, wl, dev):
@@ -239,6 +252,11 @@ def build_layers(torch, w4, prep, wl, dev):
     packed = []
     for i, (name, K, N) in enumerate(wl["linears"]):
         X, Xc, W, bias = device_linear_inputs(torch, wl, K, N, wl["seed"] + 100 * i, dev)
+        if name in wl["swiglu"]:
+            # the kernel's row order: per 16 SwiGLU features, the gate rows then the up rows
+            order = prep.swiglu_row_order(wl["swiglu"][name], (N - wl["swiglu"][name]) // 2, device=dev)
+            W = W[order].contiguous()
+            bias = None if bias is None else bias[order].contiguous()
         pk = prep.svdquant_prepare(W, Xc, r=wl["r"], bias=bias)
         del W, Xc
         packed.append((name, K, N, X, pk))
@@ -249,7 +267,7 @@ def build_layers(torch, w4, prep, wl, dev):
                 X = X.clone()
                 pk = w4.PackedWeight(pk.Wq.clone(), pk.Wsf.clone(), pk.t_w.clone(), N, K, pk.inv_s.clone(),
                                      pk.L1t.clone(), pk.L2t.clone(), None if pk.bias is None else pk.bias.clone())
-            layers.append(Layer(torch, w4, name, wl["M"], K, N, wl["r"], X, pk, dev))
+            layers.append(Layer(torch, w4, name, wl["M"], K, N, wl["r"], X, pk, dev, wl["swiglu"].get(name)))
         sets.append(layers)
     return sets
 
@@ -313,10 +331,16 @@ def run_ours(args):
         w4.nvfp4_quantize_act(L.X, L.M, L.K, L.K, w.inv_s, w.L1t, L.r, w.t_w, L.qa.Xq, L.qa.Xsf, L.qa.t_x, L.qa.U,
                               L.ws, stream)
 
-    def gemm(L):
-        w = L.w
-        w4.w4a4_gemm(L.qa.Xq, L.qa.Xsf, L.qa.t_x, L.qa.U, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.L2t, L.r, w.bias, 0,
-                     L.Y, L.N, stream)
+    def gemm(L, qa=None, outs=None, st=None):
+        w, qa = L.w, qa or L.qa
+        Y, H = outs if outs is not None else (L.Y, L.H)
+        st = st or stream
+        if L.H is None:
+            w4.w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.L2t, L.r, w.bias, 0,
+                         Y, L.N, st)
+        else:
+            w4.w4a4_gemm_swiglu(qa.Xq, qa.Xsf, qa.t_x, qa.U, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.L2t, L.r, w.bias,
+                                L.n_plain, Y, L.n_plain, H, H.shape[1], None, None, st)
 
     def step(i, evs=None):
         for j, L in enumerate(sets[i % n_sets]):
@@ -375,10 +399,16 @@ def run_ours(args):
     # buffer set.
     layers0 = sets[0]
     xh = [L.X.cpu().pin_memory() for L in layers0]
-    yh = [[torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory() for L in layers0] for _ in range(2)]
-    bufs = [[(L.X, L.Y) for L in layers0]]
-    bufs.append([(torch.empty_like(L.X), torch.empty_like(L.Y)) for L in layers0])
-    lin_ws = [w4.new_workspace(w4.w4a4_workspace_bytes(L.M, L.N, L.K, L.r), dev) for L in layers0]
+    yh = [[[torch.empty_like(o, device="cpu").pin_memory() for o in L.outputs()] for L in layers0] for _ in range(2)]
+    bufs = [[(L.X, L.outputs()) for L in layers0]]
+    bufs.append([(torch.empty_like(L.X), [torch.empty_like(o) for o in L.outputs()]) for L in layers0])
+    # w4a4_linear (quantiser + GEMM in one call) for plain linears; for the
+    # SwiGLU projection the two public calls nvfp4_quantize_act and
+    # w4a4_gemm_swiglu, with their own activation buffers and workspace
+    lin_ws = [w4.new_workspace(w4.w4a4_workspace_bytes(L.M, L.N, L.K, L.r), dev) if L.H is None else None
+              for L in layers0]
+    e2e_qa = [None if L.H is None else
+              (Layer(torch, w4, L.name, L.M, L.K, L.N, L.r, None, L.w, dev, L.n_plain)) for L in layers0]
     s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
 
@@ -397,17 +427,23 @@ def run_ours(args):
             ev_in.record(s_in)
             s_c.wait_event(ev_in)
             if i >= 2:
-                s_c.wait_event(done_out[i - 2])       # step i-2's Y have been copied out
-            for (X, Y), L, ws in zip(b, layers0, lin_ws):
+                s_c.wait_event(done_out[i - 2])       # step i-2's outputs have been copied out
+            for (X, outs), L, ws, tmp in zip(b, layers0, lin_ws, e2e_qa):
                 w = L.w
-                w4.w4a4_linear(X, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.inv_s, w.L1t, w.L2t, L.r, w.bias, 0, Y, ws,
-                               s_c)
+                if tmp is None:
+                    w4.w4a4_linear(X, L.M, L.N, L.K, w.Wq, w.Wsf, w.t_w, w.inv_s, w.L1t, w.L2t, L.r, w.bias, 0,
+                                   outs[0], ws, s_c)
+                else:
+                    w4.nvfp4_quantize_act(X, L.M, L.K, L.K, w.inv_s, w.L1t, L.r, w.t_w, tmp.qa.Xq, tmp.qa.Xsf,
+                                          tmp.qa.t_x, tmp.qa.U, tmp.ws, s_c)
+                    gemm(L, tmp.qa, outs, s_c)
             ev_c = torch.cuda.Event()
             ev_c.record(s_c)
             s_out.wait_event(ev_c)
             with torch.cuda.stream(s_out):
-                for (_, Y), h in zip(b, yh[i % 2]):
-                    h.copy_(Y, non_blocking=True)
+                for (_, outs), hs in zip(b, yh[i % 2]):
+                    for o, h in zip(outs, hs):
+                        h.copy_(o, non_blocking=True)
             ev_out = torch.cuda.Event()
             ev_out.record(s_out)
             done_c.append(ev_c)
@@ -478,8 +514,9 @@ def run_ours(args):
                        "sampled_steps": len(sampled)},
         "e2e": {"value": round(whole_job_tflops(world, fl, 1, e2e_ms), 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": int(sum(2 * M * K for _, K, _ in wl["linears"])),
-                "d2h_bytes_per_step": int(sum(2 * M * N for _, _, N in wl["linears"])),
-                "ms_per_step": round(e2e_ms, 4), "api": "w4a4_linear", "steps": e2e_steps,
+                "d2h_bytes_per_step": int(sum(o.numel() * 2 for L in layers0 for o in L.outputs())),
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
+                "api": "w4a4_linear; nvfp4_quantize_act + w4a4_gemm_swiglu for the SwiGLU projection",
                 "pipelining": "copy-in, compute and copy-out on three streams, two buffer sets"},
         "gpu_launches": per_step_launches * args.steps,
         "gpu_launches_basis": launch_basis,
@@ -780,14 +817,19 @@ def oracle_samples(wl, n_rows, n_cols):
                         seed=wl["seed"] + 100 * i)
         p = prep.svdquant_prepare(c.w, c.x_cal, c.r, c.alpha)
         wq, wsf, tw, _ = nvfp4.quantize_activation(p["R"], None)
-        out.append((c, p, wq, wsf, tw))
+        # a SwiGLU projection's sample: half plain columns, then gate and up quarters
+        sw = (n_cols // 2, n_cols // 4) if name in wl["swiglu"] else None
+        out.append((c, p, wq, wsf, tw, sw))
     return out
 
 
 def oracle_step(samples):
     from oracle import linear as olinear
-    for c, p, wq, wsf, tw in samples:
-        olinear.w4a4_linear(c.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"], c.bias)
+    from oracle import swiglu as oswiglu
+    for c, p, wq, wsf, tw, sw in samples:
+        y, _ = olinear.w4a4_linear(c.x, p["inv_s"], wq, wsf, tw, p["L1t"], p["L2t"], c.bias)
+        if sw is not None:
+            oswiglu.split_fused(y, *sw)
 
 
 def sample_flops(wl, n_rows, n_cols):

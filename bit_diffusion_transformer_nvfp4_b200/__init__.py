@@ -21,7 +21,8 @@ __all__ = [
     "w4a4_status_string", "EPI_NONE", "EPI_GELU_TANH", "SRC_BF16", "SRC_F32",
     "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
     "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor", "w4a4_set_wait_bound",
-    "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax",
+    "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
+    "gemm_swiglu",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -46,6 +47,8 @@ _SIG = {
                              _P, _I64, _P]),
     "w4a4_gemm_next_amax": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P,
                                        _c.c_int, _P, _I64, _P, _P, _P]),
+    "w4a4_gemm_swiglu": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _I64, _P, _I64,
+                                    _P, _I64, _P, _P, _P]),
     "w4a4_linear": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _c.c_int, _P, _c.c_int, _P,
                                _P, _c.c_size_t, _P]),
     "nvfp4_quantize_act_noalloc": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P, _P]),
@@ -149,6 +152,13 @@ def w4a4_gemm_next_amax(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, ep
     _check("w4a4_gemm_next_amax", lib().w4a4_gemm_next_amax(
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), epilogue, _ptr(Y), ldy, _ptr(next_inv_s), _ptr(next_amax), _stream(stream)))
+
+
+def w4a4_gemm_swiglu(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_plain, Y, ldy, H, ldh, next_inv_s,
+                     next_amax, stream=None):
+    _check("w4a4_gemm_swiglu", lib().w4a4_gemm_swiglu(
+        _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
+        _ptr(bias), n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s), _ptr(next_amax), _stream(stream)))
 
 
 def w4a4_linear(X, M, N, K, Wq, Wsf, t_w, inv_s, L1t, L2t, r, bias, epilogue, Y, workspace, stream=None):
@@ -281,6 +291,23 @@ def gemm(qa: QuantizedActivation, w: PackedWeight, epilogue: int = EPI_NONE, Y=N
         w4a4_gemm_next_amax(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias,
                             epilogue, Y, Y.stride(0), next_inv_s, next_amax, stream)
     return Y
+
+
+def gemm_swiglu(qa: QuantizedActivation, w: PackedWeight, n_plain: int, Y=None, H=None, stream=None,
+                next_inv_s=None, next_amax=None):
+    """The fused projection with the SwiGLU epilogue: the first ``n_plain``
+    packed weight rows give Y [M, n_plain]; the rest, gate/up pairs in the
+    order of ``prep.swiglu_row_order``, give H = silu(gate) * up [M, (N -
+    n_plain) / 2].  Returns (Y, H)."""
+    n_h = (w.N - n_plain) // 2
+    dev = qa.Xq.device
+    if Y is None and n_plain > 0:
+        Y = torch.empty(qa.M, n_plain, dtype=torch.bfloat16, device=dev)
+    if H is None:
+        H = torch.empty(qa.M, n_h, dtype=torch.bfloat16, device=dev)
+    w4a4_gemm_swiglu(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias, n_plain,
+                     Y, Y.stride(0) if Y is not None else 0, H, H.stride(0), next_inv_s, next_amax, stream)
+    return Y, H
 
 
 def linear(X: torch.Tensor, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, workspace=None, stream=None):

@@ -54,6 +54,15 @@ struct GemmParams {
   // null (all ones).
   const float* next_inv_s;
   unsigned* next_amax;
+  // SwiGLU epilogue (CTA-pair kernel only): weight rows [0, n_plain) give
+  // plain outputs in Y; rows [n_plain, N) hold gate/up pairs in blocks of 32
+  // (16 gate rows, then the 16 up rows of the same features), and the
+  // kernel writes silu(gate) * up of each pair to H [M, (N - n_plain) / 2]
+  // (row stride ldh).  n_plain == N: no SwiGLU columns.  With next_amax the
+  // amax covers H only.
+  int n_plain;
+  __nv_bfloat16* H;
+  int64_t ldh;
 };
 
 // Shared-memory descriptors of the low-rank pass, K step k (16 columns) of
@@ -142,6 +151,16 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ float gelu_tanh_f32(float y) {
   const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
   const float t = ex2_approx(-2.8853900817779268f * fabsf(u));  // exp(-2|u|) = 2^(-2 log2(e) |u|)
+  const float num = y < 0.0f ? y * t : y;
+  return num * rcp_approx(1.0f + t);
+}
+
+// silu(y) = y sigmoid(y).  With t = exp(-|y|) in (0, 1] it equals y / (1 + t)
+// for y >= 0 and y t / (1 + t) for y < 0: no overflow (t underflows to 0 for
+// large |y|, giving y and -0) and no IEEE division; the hardware base-2
+// exponential and reciprocal keep it within a few fp32 ulps.
+__device__ __forceinline__ float silu_f32(float y) {
+  const float t = ex2_approx(-1.4426950408889634f * fabsf(y));  // exp(-|y|) = 2^(-log2(e) |y|)
   const float num = y < 0.0f ? y * t : y;
   return num * rcp_approx(1.0f + t);
 }

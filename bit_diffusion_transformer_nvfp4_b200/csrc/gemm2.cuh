@@ -100,7 +100,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                  const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_l2,
-                 const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_h,
+                 const GemmParams p) {
   constexpr int BN = C::BN, STAGES = C::STAGES;
   // the next kernel in the stream (a programmatic dependent) may be scheduled
   // on SMs this grid leaves; it waits for this grid's completion itself
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tma_prefetch_desc(&tm_sfa);
     tma_prefetch_desc(&tm_sfb);
     tma_prefetch_desc(&tm_y);
+    if (p.n_plain < p.N) tma_prefetch_desc(&tm_h);
     if (lr) {
       tma_prefetch_desc(&tm_u);
       tma_prefetch_desc(&tm_l2);
@@ -354,78 +356,142 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * acc);
 
       const int row0 = m0 + q * 32;
-#pragma unroll
-      for (int c = 0; c < C::HALF / 32; ++c, ++chunk) {
-        const int n = n0 + h * C::HALF + 32 * c;
+      // the staging buffer of the next 32 x 32 output box, once the TMA store
+      // that last used it has finished reading it
+      auto next_buf = [&]() -> uint8_t* {
         uint8_t* buf = stage_buf + (chunk % C::EPI_NBUF) * C::EPI_BUF;
         if (chunk >= static_cast<uint32_t>(C::EPI_NBUF)) {
-          // the TMA store that last used this buffer has finished reading it
           if (lane == 0) bulk_wait_group_read<C::EPI_NBUF - 1>();
           __syncwarp();
         }
-        uint32_t packed[16];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float b[8];
-          if (p.bias != nullptr && n + 8 * g < p.N) {
-            const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8 * g));
-            b[0] = bf16_lo(bw.x); b[1] = bf16_hi(bw.x); b[2] = bf16_lo(bw.y); b[3] = bf16_hi(bw.y);
-            b[4] = bf16_lo(bw.z); b[5] = bf16_hi(bw.z); b[6] = bf16_lo(bw.w); b[7] = bf16_hi(bw.w);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) b[j] = 0.0f;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            float y0 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j])), b[j]);
-            float y1 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j + 1])), b[j + 1]);
-            if (p.epi == 1) {
-              y0 = gelu_tanh_f32(y0);
-              y1 = gelu_tanh_f32(y1);
-            }
-            packed[4 * g + j / 2] = pack_bf16x2(y0, y1);
-          }
-        }
-        // row `lane` of a 32 x 32 bf16 box, 64-byte rows, 64-byte swizzle
+        return buf;
+      };
+      // row `lane` of a 32 x 32 bf16 box, 64-byte rows, 64-byte swizzle
+      auto stage_row = [&](uint8_t* buf, const uint32_t (&packed)[16]) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int phys = g ^ ((lane >> 1) & 3);
           *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
               make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
         }
-        if (p.next_amax != nullptr) {
-          // next layer's amax over the staged chunk (only outputs the TMA
-          // store keeps: rows < M, columns < N).  Lane l takes columns 2(l%16),
-          // 2(l%16)+1 of rows 16(l/16) .. +15: packed maxima of |y| down the
-          // column pair, then one multiply by the next 1/s per column.
-          __syncwarp();
-          const int cpair = lane & 15;
-          const int rbase = (lane >> 4) * 16;
-          uint32_t mx = 0u;
+      };
+      // next layer's amax over a staged box (only outputs the TMA store
+      // keeps: rows < M, columns < ncols).  Lane l takes columns 2(l%16),
+      // 2(l%16)+1 of rows 16(l/16) .. +15: packed maxima of |y| down the
+      // column pair, then one multiply by the next 1/s per column.
+      auto fold_amax = [&](const uint8_t* buf, int col0, int ncols) {
+        __syncwarp();
+        const int cpair = lane & 15;
+        const int rbase = (lane >> 4) * 16;
+        uint32_t mx = 0u;
 #pragma unroll
-          for (int rr = 0; rr < 16; ++rr) {
-            const int row = rbase + rr;
-            if (row0 + row < p.M) {
-              const int phys = (cpair >> 2) ^ ((row >> 1) & 3);
-              mx = bf16x2_absmax(mx, *reinterpret_cast<const uint32_t*>(buf + row * 64 + phys * 16 + (cpair & 3) * 4));
-            }
-          }
-          const int col = n + 2 * cpair;
-          if (col < p.N) {  // N % 8 == 0: both columns of the pair are valid
-            float v0 = bf16_lo(mx & 0x7FFF7FFFu), v1 = bf16_hi(mx & 0x7FFF7FFFu);
-            if (p.next_inv_s != nullptr) {
-              const float2 s2 = __ldg(reinterpret_cast<const float2*>(p.next_inv_s + col));
-              v0 = __fmul_rn(v0, s2.x);
-              v1 = __fmul_rn(v1, s2.y);
-            }
-            amax = fmaxf(amax, fmaxf(v0, v1));
+        for (int rr = 0; rr < 16; ++rr) {
+          const int row = rbase + rr;
+          if (row0 + row < p.M) {
+            const int phys = (cpair >> 2) ^ ((row >> 1) & 3);
+            mx = bf16x2_absmax(mx, *reinterpret_cast<const uint32_t*>(buf + row * 64 + phys * 16 + (cpair & 3) * 4));
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_y, smem_u32(buf), n, row0);
-          bulk_commit_group();
+        const int col = col0 + 2 * cpair;
+        if (col < ncols) {  // ncols % 8 == 0: both columns of the pair are valid
+          float v0 = bf16_lo(mx & 0x7FFF7FFFu), v1 = bf16_hi(mx & 0x7FFF7FFFu);
+          if (p.next_inv_s != nullptr) {
+            const float2 s2 = __ldg(reinterpret_cast<const float2*>(p.next_inv_s + col));
+            v0 = __fmul_rn(v0, s2.x);
+            v1 = __fmul_rn(v1, s2.y);
+          }
+          amax = fmaxf(amax, fmaxf(v0, v1));
+        }
+      };
+      if (n0 < p.n_plain) {
+        // ---------------------------------------------------- plain outputs
+#pragma unroll
+        for (int c = 0; c < C::HALF / 32; ++c, ++chunk) {
+          const int n = n0 + h * C::HALF + 32 * c;
+          uint8_t* buf = next_buf();
+          uint32_t packed[16];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float b[8];
+            if (p.bias != nullptr && n + 8 * g < p.n_plain) {
+              const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8 * g));
+              b[0] = bf16_lo(bw.x); b[1] = bf16_hi(bw.x); b[2] = bf16_lo(bw.y); b[3] = bf16_hi(bw.y);
+              b[4] = bf16_lo(bw.z); b[5] = bf16_hi(bw.z); b[6] = bf16_lo(bw.w); b[7] = bf16_hi(bw.w);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) b[j] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              float y0 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j])), b[j]);
+              float y1 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j + 1])), b[j + 1]);
+              if (p.epi == 1) {
+                y0 = gelu_tanh_f32(y0);
+                y1 = gelu_tanh_f32(y1);
+              }
+              packed[4 * g + j / 2] = pack_bf16x2(y0, y1);
+            }
+          }
+          stage_row(buf, packed);
+          if (p.next_amax != nullptr && p.n_plain == p.N) fold_amax(buf, n, p.N);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_y, smem_u32(buf), n, row0);
+            bulk_commit_group();
+          }
+        }
+      } else {
+        // ---------------------------------------------------- SwiGLU pairs
+        // Each 32-column accumulator block holds 16 gate and then the 16 up
+        // features of the same outputs; two blocks fill one 32-column box of H.
+        const int n_h = (p.N - p.n_plain) / 2;
+        const int hc0 = (n0 - p.n_plain) / 2 + h * (C::HALF / 2);
+#pragma unroll
+        for (int c2 = 0; c2 < C::HALF / 64; ++c2, ++chunk) {
+          uint8_t* buf = next_buf();
+          uint32_t packed[16];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int c = 2 * c2 + hh;
+            const int nw = n0 + h * C::HALF + 32 * c;  // first gate row of the block
+            float bg[16], bu[16];
+            if (p.bias != nullptr && nw < p.N) {  // (N - n_plain) % 32 == 0: the whole block is valid
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                const uint4 gw = __ldg(reinterpret_cast<const uint4*>(p.bias + nw + 8 * v));
+                const uint4 uw = __ldg(reinterpret_cast<const uint4*>(p.bias + nw + 16 + 8 * v));
+                const uint32_t gg[4] = {gw.x, gw.y, gw.z, gw.w}, uu[4] = {uw.x, uw.y, uw.z, uw.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  bg[8 * v + 2 * j] = bf16_lo(gg[j]);
+                  bg[8 * v + 2 * j + 1] = bf16_hi(gg[j]);
+                  bu[8 * v + 2 * j] = bf16_lo(uu[j]);
+                  bu[8 * v + 2 * j + 1] = bf16_hi(uu[j]);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) bg[j] = bu[j] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+              const float g0 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + j])), bg[j]);
+              const float g1 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + j + 1])), bg[j + 1]);
+              const float u0 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 16 + j])), bu[j]);
+              const float u1 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 16 + j + 1])), bu[j + 1]);
+              packed[8 * hh + j / 2] = pack_bf16x2(__fmul_rn(silu_f32(g0), u0), __fmul_rn(silu_f32(g1), u1));
+            }
+          }
+          stage_row(buf, packed);
+          const int hc = hc0 + 32 * c2;
+          if (p.next_amax != nullptr) fold_amax(buf, hc, n_h);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_h, smem_u32(buf), hc, row0);
+            bulk_commit_group();
+          }
         }
       }
       ++tcount;

@@ -418,6 +418,9 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   p.status = dev->status_ptr;
   p.next_inv_s = next_inv_s;
   p.next_amax = next_amax;
+  p.n_plain = static_cast<int>(N);
+  p.H = nullptr;
+  p.ldh = 0;
   const int64_t tiles = ceil_div(M, C::BM) * ceil_div(N, C::BN);
   const int64_t grid = tiles < dev->num_sms ? tiles : dev->num_sms;
   cudaLaunchConfig_t cfg = {};
@@ -442,8 +445,12 @@ template <class C>
 int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                      int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
                      const void* bias, int epi, void* Y, int64_t ldy, const float* next_inv_s, unsigned* next_amax,
-                     cudaStream_t stream, DeviceInfo* dev) {
-  CUtensorMap ta, tb, tsa, tsb, tu, tl, ty;
+                     cudaStream_t stream, DeviceInfo* dev, int64_t n_plain = -1, void* H = nullptr,
+                     int64_t ldh = 0) {
+  if (n_plain < 0) n_plain = N;
+  // SwiGLU outputs fill 32-column boxes from two 32-column accumulator blocks
+  if (n_plain < N && (C::BN % 64 != 0 || n_plain % C::BN != 0)) return W4A4_ERR_SHAPE;
+  CUtensorMap ta, tb, tsa, tsb, tu, tl, ty, th;
   if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(K / 2), 128u, 128u, CU_TENSOR_MAP_SWIZZLE_128B))
     return W4A4_ERR_CUDA;
@@ -452,9 +459,20 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
     return W4A4_ERR_CUDA;
   if (!encode_sf(&tsa, Xsf, M, K, 1)) return W4A4_ERR_CUDA;
   if (!encode_sf(&tsb, Wsf, N, K, static_cast<uint32_t>(C::SFB_RB))) return W4A4_ERR_CUDA;
-  if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
-                 static_cast<uint64_t>(ldy) * 2, 32u, 32u, CU_TENSOR_MAP_SWIZZLE_64B))
+  // plain outputs Y [M, n_plain] and SwiGLU outputs H [M, (N - n_plain) / 2],
+  // both written in 32 x 32 boxes
+  if (n_plain > 0 && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(n_plain),
+                                static_cast<uint64_t>(M), static_cast<uint64_t>(ldy) * 2, 32u, 32u,
+                                CU_TENSOR_MAP_SWIZZLE_64B))
     return W4A4_ERR_CUDA;
+  if (n_plain < N) {
+    if (!encode_2d(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, static_cast<uint64_t>((N - n_plain) / 2),
+                   static_cast<uint64_t>(M), static_cast<uint64_t>(ldh) * 2, 32u, 32u, CU_TENSOR_MAP_SWIZZLE_64B))
+      return W4A4_ERR_CUDA;
+    if (n_plain == 0) ty = th;  // unused
+  } else {
+    th = ty;  // unused
+  }
   if (r > 0) {
     // U = [hi | lo], rows of 2r bf16; L2t rows of r bf16 (swizzle = row width)
     if (!encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, U, static_cast<uint64_t>(2 * r), static_cast<uint64_t>(M),
@@ -484,6 +502,9 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   p.status = dev->status_ptr;
   p.next_inv_s = next_inv_s;
   p.next_amax = next_amax;
+  p.n_plain = static_cast<int>(n_plain);
+  p.H = static_cast<__nv_bfloat16*>(H);
+  p.ldh = ldh;
   const int64_t tiles = ceil_div(M, 2 * C::BM) * ceil_div(N, C::BN);
   const int64_t max_pairs = dev->num_sms / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -501,7 +522,7 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, gemm2_kernel<C>, ta, tb, tsa, tsb, tu, tl, ty, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, gemm2_kernel<C>, ta, tb, tsa, tsb, tu, tl, ty, th, p) != cudaSuccess) {
     cudaGetLastError();
     return W4A4_ERR_CUDA;
   }
@@ -655,6 +676,29 @@ int w4a4_gemm_next_amax(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x,
     return W4A4_ERR_ALIGN;
   return gemm_dispatch(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy, next_inv_s,
                        reinterpret_cast<unsigned*>(next_amax), stream);
+}
+
+int w4a4_gemm_swiglu(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                     int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                     const void* bias, int64_t n_plain, void* Y, int64_t ldy, void* H, int64_t ldh,
+                     const float* next_inv_s, float* next_amax, void* stream) {
+  if (n_plain < 0 || n_plain >= N || n_plain % 256 != 0 || (N - n_plain) % 32 != 0) return W4A4_ERR_SHAPE;
+  const int64_t n_h = (N - n_plain) / 2;
+  if (ldh < n_h || ldh % 8 != 0 || (n_plain > 0 && (ldy < n_plain || ldy % 8 != 0))) return W4A4_ERR_SHAPE;
+  // the common checks, with the plain part's columns standing for Y's
+  int st = check_gemm_args(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, W4A4_EPI_NONE,
+                           n_plain > 0 ? Y : H, N);
+  if (st != W4A4_OK || M == 0) return st;
+  if (!H || (n_plain > 0 && !Y)) return W4A4_ERR_NULL;
+  if (!aligned16(H) || (n_plain > 0 && !aligned16(Y)) || (next_inv_s && !aligned16(next_inv_s)) ||
+      reinterpret_cast<uintptr_t>(next_amax) % 4 != 0)
+    return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  return launch_gemm_pair<PairMain>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, W4A4_EPI_NONE, Y, ldy,
+                                    next_inv_s, reinterpret_cast<unsigned*>(next_amax),
+                                    static_cast<cudaStream_t>(stream), dev, n_plain, H, ldh);
 }
 
 int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,

@@ -54,3 +54,20 @@ def svdquant_prepare(w: torch.Tensor, x_cal: torch.Tensor, r: int = 32, alpha: f
     packed = pack_weight(resid, inv_s=inv_s, L1t=L1t, L2t=L2t,
                          bias=None if bias is None else bias.to(torch.bfloat16).contiguous())
     return packed
+
+
+def swiglu_row_order(n_plain: int, n_ff: int, device=None) -> torch.Tensor:
+    """Row order that ``w4a4_gemm_swiglu`` expects for a fused projection
+    whose weight is laid out [plain (n_plain rows) | gate (n_ff) | up (n_ff)]:
+    the plain rows, then per block of 16 features its 16 gate rows followed
+    by its 16 up rows.  Apply it to the weight (and bias) before
+    ``svdquant_prepare``: a row permutation leaves the smoothing factors and
+    the singular values unchanged and permutes the residual and L2t rows."""
+    if n_ff % 16:
+        raise ValueError("n_ff must be a multiple of 16")
+    blocks = torch.arange(n_ff // 16, device=device)[:, None]
+    i = torch.arange(16, device=device)[None, :]
+    gate = n_plain + 16 * blocks + i
+    up = n_plain + n_ff + 16 * blocks + i
+    tail = torch.cat([gate, up], dim=1).reshape(-1)
+    return torch.cat([torch.arange(n_plain, device=device), tail])

@@ -230,6 +230,39 @@ int w4a4_gemm_next_amax(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x,
                         void* stream);
 
 /*
+ * w4a4_gemm_swiglu -- w4a4_gemm for a fused projection whose last output
+ * features are SwiGLU gate/up pairs: the kernel applies the SwiGLU epilogue
+ * that the NVIDIA blog page on FLUX on Blackwell fuses into its NVFP4 GEMM
+ * ("NVIDIA Technical Blog Details FLUX 3 Image Klein Blackwell Inference
+ * Optimization Methods", the NVFP4 / fused-GEMM paragraph), so the gate and
+ * up features never reach memory.  With y[m,n] = t_x t_w acc[m,n] + bias[n]
+ * in fp32 (acc as in w4a4_gemm, over the packed weight rows n):
+ *   rows n < n_plain:   Y[m,n] = bf16(y[m,n])
+ *   rows n >= n_plain:  grouped in blocks of 32, block b = 16 gate rows
+ *                       n_plain + 32b + i and then the 16 up rows
+ *                       n_plain + 32b + 16 + i (i = 0..15) of output
+ *                       features j = 16b + i:
+ *                       H[m,j] = bf16(silu(y[m, gate row]) * y[m, up row]),
+ *                       silu(v) = v / (1 + exp(-v))
+ * (the Python package's prep.swiglu_row_order gives the row order for a weight laid
+ * out [plain | gate | up]).  Same arguments as w4a4_gemm, without epilogue,
+ * plus
+ *   n_plain     plain output features, a multiple of 256, 0 <= n_plain < N;
+ *               (N - n_plain) a multiple of 32
+ *   Y, ldy      bf16 [M, ldy], ldy >= n_plain (Y may be NULL iff n_plain == 0)
+ *   H, ldh      bf16 [M, ldh], ldh >= (N - n_plain) / 2, ldh % 8 == 0
+ *   next_inv_s, next_amax  as in w4a4_gemm_next_amax, over H only (the next
+ *               layer's input; next_inv_s indexed by H's column), or
+ *               next_amax NULL for none
+ * Launches one CTA-pair GEMM kernel.
+ */
+int w4a4_gemm_swiglu(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U,
+                     int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,
+                     const float* t_w, const void* L2t, int r, const void* bias, int64_t n_plain,
+                     void* Y, int64_t ldy, void* H, int64_t ldh, const float* next_inv_s,
+                     float* next_amax, void* stream);
+
+/*
  * w4a4_linear -- the whole hot path: nvfp4_quantize_act on X (row stride K)
  * into the workspace, then w4a4_gemm into Y (row stride N).
  *   workspace >= w4a4_workspace_bytes(M, N, K, r) bytes of device memory.

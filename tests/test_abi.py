@@ -189,3 +189,18 @@ def test_wait_bound_argument_check(so):
     assert so.w4a4_set_wait_bound(5) == -8
     if not __import__("torch").cuda.is_available():
         assert so.w4a4_set_wait_bound(0) == -4
+
+
+def test_swiglu_argument_checks(so):
+    """w4a4_gemm_swiglu rejects bad splits, strides and pointers on the host."""
+    P = 1 << 20
+    f = so.w4a4_gemm_swiglu
+    #        Xq Xsf t_x U     M    N     K    Wq Wsf t_w L2t  r  bias n_plain Y  ldy H  ldh  s     amax  stream
+    assert f(P, P, P, None, 128, 1024, 512, P, P, P, None, 0, None, 128, P, 128, P, 448, None, None, None) == -2
+    assert f(P, P, P, None, 128, 1024, 512, P, P, P, None, 0, None, 256, P, 256, P, 368, None, None, None) == -2
+    assert f(P, P, P, None, 128, 1040, 512, P, P, P, None, 0, None, 256, P, 256, P, 392, None, None, None) == -2
+    assert f(P, P, P, None, 128, 1024, 512, P, P, P, None, 0, None, 1024, P, 1024, P, 8, None, None, None) == -2
+    assert f(P, P, P, None, 128, 1024, 512, P, P, P, None, 0, None, 256, P, 256, None, 384, None, None, None) == -1
+    assert f(P, P, P, None, 128, 1024, 512, P, P, P, None, 0, None, 256, P, 256, P + 2, 384, None, None, None) == -3
+    assert f(None, None, None, None, 0, 1024, 512, None, None, None, None, 0, None, 256, None, 256, None, 384,
+             None, None, None) == 0

@@ -120,3 +120,55 @@ def test_config4_ragged_rows(w4, layers, which):
     y_ref, aux = olinear.w4a4_linear(x, p["inv_s"], owq, osf, ot, p["L1t"], p["L2t"][cols],
                                      None if c.bias is None else c.bias[cols], rows=rows)
     check_y(y, y_ref)
+
+
+def test_config4_swiglu_full_size(w4, layers):
+    """The fused projection as the block runs it: QKV (3 x 6144 plain
+    features) and SwiGLU (18432 gate/up pairs) in one GEMM at 16896 tokens,
+    the kernel's row order from prep.swiglu_row_order; sampled Y and H
+    against the oracle in the natural order, and the epilogue's amax over H
+    (the output linear's input) as a property of the whole stored H."""
+    import torch
+    from bit_diffusion_transformer_nvfp4_b200 import prep as gprep
+    from oracle import swiglu as oswiglu
+    c, p, _ = layers[0]
+    n_plain = n_ff = 18432
+    assert c.N == n_plain + 2 * n_ff
+    perm = gprep.swiglu_row_order(n_plain, n_ff).numpy()
+    pw = w4.pack_weight(to_dev_f32(p["R"][perm]))
+    w = w4.PackedWeight(pw.Wq, pw.Wsf, pw.t_w, c.N, c.K, to_dev_f32(p["inv_s"]), to_dev_bf16(p["L1t"]),
+                        to_dev_bf16(p["L2t"][perm]), None)
+    qa = w4.quantize_act(to_dev_bf16(c.x), w.inv_s, w.L1t, w.t_w)
+    s_next = (1.0 / np.exp(0.3 * rng(44).standard_normal(n_ff))).astype(np.float32)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    Y, H = w4.gemm_swiglu(qa, w, n_plain, next_inv_s=to_dev_f32(s_next), next_amax=amax)
+    torch.cuda.synchronize()
+    assert w4.w4a4_device_status() == 0
+
+    g = rng(45)
+    rows = np.sort(g.choice(c.M, 64, replace=False))
+    rows[-1] = c.M - 1
+    pc = np.sort(g.choice(n_plain, 128, replace=False))
+    hc = np.sort(g.choice(n_ff, 128, replace=False))
+    hc[-1] = n_ff - 1
+    cols = np.concatenate([pc, n_plain + hc, n_plain + n_ff + hc])      # natural order
+    # the GPU's packing of these rows (kernel order) is the oracle's
+    oq, osf, ot = nvfp4.quantize(p["R"][cols], amax=np.max(np.abs(p["R"])))
+    inv = np.argsort(perm)                                                # natural row -> kernel row
+    assert float(pw.t_w.cpu()[0]) == float(ot)
+    np.testing.assert_array_equal(pw.Wq.cpu().numpy()[inv[cols]], nvfp4.pack(oq))
+    np.testing.assert_array_equal(sf_atoms_to_rowmajor(pw.Wsf.cpu().numpy(), c.N, c.K)[inv[cols]], osf)
+    y_ref, _ = olinear.w4a4_linear(c.x, p["inv_s"], nvfp4.pack(oq), osf, ot, p["L1t"], p["L2t"][cols], None,
+                                   rows=rows)
+    plain_ref = y_ref[:, :len(pc)]
+    h_ref = oswiglu.swiglu(y_ref[:, len(pc):len(pc) + len(hc)], y_ref[:, len(pc) + len(hc):])
+    idx = torch.from_numpy(rows).cuda()
+    check_y(from_dev_bf16(Y[idx])[:, pc], plain_ref)
+    check_y(from_dev_bf16(H[idx])[:, hc], h_ref)
+
+    got = float(amax.cpu()[0])
+    want = np.float32(0.0)
+    for r0 in range(0, c.M, 2048):
+        h = from_dev_bf16(H[r0:r0 + 2048])
+        want = max(want, np.float32(np.max(np.abs((h * s_next[None, :]).astype(np.float32)))))
+    assert got == float(want)
