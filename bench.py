@@ -175,6 +175,7 @@ class ClockSampler:
     def summarise(rows, sm_floor=300.0):
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         sm = []
+        power = []
         reasons = set()
         max_mhz = None
         for r in rows:
@@ -186,11 +187,16 @@ class ClockSampler:
             if mhz < sm_floor:
                 continue
             sm.append(mhz)
+            try:
+                power.append(float(r[3]))
+            except ValueError:
+                pass
             for n, v in zip(names, r[4:]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max_mhz,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": statistics.median(power) if power else None}
 
 
 # ---------------------------------------------------------------- our arm
@@ -478,9 +484,11 @@ def run_ours(args):
         ach = g_fl / (gemm_ms[j] * 1e-3) / 1e12
         a0, a = quant_bytes(M, K, r)
         qach = (a0 + a) / (quant_ms[j] * 1e-3) / 1e9
+        # the GEMM is timed inside a seconds-long loop of steps, as the
+        # sustained bf16 figure was measured: its FP4 equivalent is the peak
         rooflines.append({"kernel": f"gemm2_kernel ({name})", "bound": "tensor", "achieved": round(ach, 2),
-                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(ach / fp4_peak, 4),
-                          "frac_of_sustained": round(ach / fp4_peak_sus, 4), "launch_ms": round(gemm_ms[j], 5),
+                          "peak": round(fp4_peak_sus, 1), "unit": "TFLOP/s", "frac": round(ach / fp4_peak_sus, 4),
+                          "frac_of_burst": round(ach / fp4_peak, 4), "launch_ms": round(gemm_ms[j], 5),
                           "algorithmic_flops_per_launch": g_fl})
         rooflines.append({"kernel": f"activation quantiser ({name}: tensor amax + quantise pass)", "bound": "hbm",
                           "achieved": round(qach, 1), "peak": hbm, "unit": "GB/s", "frac": round(qach / hbm, 4),
@@ -489,8 +497,10 @@ def run_ours(args):
     top = max(range(n_lin), key=lambda j: gemm_ms[j])
     dom = dict(rooflines[2 * top])
     dom["traffic"] = ncu_traffic(GEMM_SOURCES, GEMM_SUMMARY[args.workload]) if top == 0 else None
-    dom["peak_kind"] = (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_OVER_BF16:g} (nominal "
-                        f"FP4/BF16 ratio); frac_of_sustained uses the sustained bf16 figure x {FP4_OVER_BF16:g}")
+    dom["peak_kind"] = (f"{peak_kind} sustained bf16 {peaks.get('bf16_tflops_sustained')} TFLOP/s x "
+                        f"{FP4_OVER_BF16:g} (nominal FP4/BF16 ratio): the kernel runs inside a seconds-long loop "
+                        f"under the power cap; frac_of_burst uses the burst figure {peaks['bf16_tflops']} x "
+                        f"{FP4_OVER_BF16:g}")
     clocks = ClockSampler.summarise(clock_rows)
     if per_step_launches is None:
         per_step_launches = sum(1 + (2 if 2 * M * K > 64 << 20 else 1) for _, K, _n in wl["linears"])
@@ -504,9 +514,13 @@ def run_ours(args):
         "data": "synthetic (seeded, drawn on the GPU)",
         "config": dict(workload_config(args.workload),
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU", l2=wl["l2"]),
-        "pct_fp4_peak": round(100.0 * value / (world * fp4_peak), 2),
-        "fp4_peak_tflops": round(fp4_peak, 1),
-        "fp4_peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOPS x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)",
+        "pct_fp4_peak": round(100.0 * value / (world * fp4_peak_sus), 2),
+        "pct_fp4_peak_burst": round(100.0 * value / (world * fp4_peak), 2),
+        "fp4_peak_tflops": round(fp4_peak_sus, 1),
+        "fp4_peak_burst_tflops": round(fp4_peak, 1),
+        "fp4_peak_basis": (f"{peak_kind} sustained bf16 {peaks.get('bf16_tflops_sustained')} TFLOPS x "
+                           f"{FP4_OVER_BF16:g} (nominal FP4/BF16 ratio); burst {peaks['bf16_tflops']} x "
+                           f"{FP4_OVER_BF16:g}"),
         "roofline": dom,
         "rooflines": rooflines,
         "kernels_ms": {**{f"quant_{n}": round(quant_ms[j], 5) for j, (n, _, _) in enumerate(wl["linears"])},
@@ -793,6 +807,99 @@ def run_table(args):
         torch.cuda.empty_cache()
 
 
+# ---------------------------------------------------------------- profiling cases
+
+CASES = {
+    # name: (what, M, K, N or None, extra)
+    "gemm_block2048_up": ("w4a4_gemm_swiglu, the 2048px fused QKV+SwiGLU-up projection", 16896, 6144, 55296, 18432),
+    "gemm_block2048_up_small": ("w4a4_gemm_swiglu, the 2048px fused projection at 4096 tokens", 4096, 6144, 55296, 18432),
+    "gemm_block2048_out": ("w4a4_gemm, the 2048px output projection", 16896, 24576, 6144, None),
+    "gemm_flux1024_qkv": ("w4a4_gemm, the FLUX-1024px QKV projection (CTA pairs, 256 x 256 tiles)", 4608, 3072, 9216, None),
+    "gemm_row_block": ("w4a4_gemm on a single 128-row block (CTA pairs, 256 x 64 tiles)", 128, 3072, 3072, None),
+    "gemm_single_cta": ("w4a4_gemm on a single row block with N > 64 SMs (single-CTA 128 x 192 tiles)", 64, 3072, 19200,
+                        None),
+    "quant_fused_flux1024": ("nvfp4_quantize_act, single pass (4608 x 3072)", 4608, 3072, None, None),
+    "quant_two_pass_block2048": ("nvfp4_quantize_act, two passes (16896 x 6144)", 16896, 6144, None, None),
+    "quant_stream_block2048": ("nvfp4_quantize_act_with_amax, streaming pass (16896 x 6144)", 16896, 6144, None, None),
+    "pack_weight_block2048_out": ("nvfp4_pack_weight on an fp32 residual (6144 x 24576)", 6144, 24576, None, None),
+}
+
+
+def run_case(args):
+    """One kernel's small workload for an ncu capture: ``--steps`` calls of the
+    entry point after ``--warmup`` untimed ones, inputs drawn on the GPU
+    (lognormal channel magnitudes), rank 32.  Prints the mean event time per
+    call.  Nothing here is a benchmark line."""
+    import torch
+    import bit_diffusion_transformer_nvfp4_b200 as w4
+    what, M, K, N, n_plain = CASES[args.case]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w4.lib()
+    st = torch.cuda.current_stream()
+    g = torch.Generator(device=dev)
+    g.manual_seed(77)
+    r = 32
+    mags = torch.exp(1.5 * torch.randn(K, generator=g, device=dev))
+    inv_s = (1.0 / torch.exp(0.3 * torch.randn(K, generator=g, device=dev))).contiguous()
+    L1t = (0.02 * torch.randn(r, K, generator=g, device=dev)).to(torch.bfloat16)
+    t_w = torch.full((1,), 0.01, device=dev)
+    if args.case.startswith("pack_weight"):
+        R = 0.02 * torch.randn(M, K, generator=g, device=dev)
+        ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, 0), dev)
+        Wq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        Wsf = torch.empty(w4.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev)
+        tw = torch.empty(1, device=dev)
+
+        def call():
+            w4.nvfp4_pack_weight(R, w4.SRC_F32, M, K, K, Wq, Wsf, tw, ws, st)
+    else:
+        X = (torch.randn(M, K, generator=g, device=dev) * mags).to(torch.bfloat16)
+        qa = w4.quantize_act(X, inv_s, L1t, t_w)
+        ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
+        amax = torch.full((1,), float((X.float() * inv_s).abs().max()), device=dev)
+        if args.case.startswith("quant_stream"):
+            def call():
+                w4.nvfp4_quantize_act_with_amax(X, M, K, K, inv_s, L1t, r, t_w, amax, qa.Xq, qa.Xsf, qa.t_x, qa.U,
+                                                ws, st)
+        elif args.case.startswith("quant"):
+            def call():
+                w4.nvfp4_quantize_act(X, M, K, K, inv_s, L1t, r, t_w, qa.Xq, qa.Xsf, qa.t_x, qa.U, ws, st)
+        else:
+            W = 0.02 * torch.randn(N, K, generator=g, device=dev)
+            pw = w4.pack_weight(W)
+            del W
+            L2t = (0.02 * torch.randn(N, r, generator=g, device=dev)).to(torch.bfloat16)
+            if n_plain is None:
+                Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+                def call():
+                    w4.w4a4_gemm(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, pw.Wq, pw.Wsf, pw.t_w, L2t, r, None, 0, Y, N,
+                                 st)
+            else:
+                Y = torch.empty(M, n_plain, dtype=torch.bfloat16, device=dev)
+                H = torch.empty(M, (N - n_plain) // 2, dtype=torch.bfloat16, device=dev)
+
+                def call():
+                    w4.w4a4_gemm_swiglu(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, pw.Wq, pw.Wsf, pw.t_w, L2t, r, None,
+                                        n_plain, Y, n_plain, H, H.shape[1], None, None, st)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        call()
+    e1.record(st)
+    torch.cuda.synchronize()
+    status = w4.w4a4_device_status()
+    print(json.dumps({"case": args.case, "what": what, "M": M, "K": K, "N": N, "calls": args.steps,
+                      "warmup": args.warmup, "us_per_call": round(e0.elapsed_time(e1) / args.steps * 1e3, 2),
+                      "status": status}), flush=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+
 # ---------------------------------------------------------------- oracle arms
 
 def cpu_threads():
@@ -903,10 +1010,14 @@ def main():
     ap.add_argument("--table", action="store_true",
                     help="time every configuration's layers (one JSON line per row) instead of the benchmark step")
     ap.add_argument("--table-reps", type=int, default=20)
+    ap.add_argument("--case", choices=sorted(CASES),
+                    help="run one kernel's small profiling workload (--steps calls after --warmup) instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.table:
+    if args.case:
+        run_case(args)
+    elif args.table:
         run_table(args)
     elif args.impl == "reference":
         run_reference(args)

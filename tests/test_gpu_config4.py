@@ -153,7 +153,7 @@ def test_config4_swiglu_full_size(w4, layers):
     hc[-1] = n_ff - 1
     cols = np.concatenate([pc, n_plain + hc, n_plain + n_ff + hc])      # natural order
     # the GPU's packing of these rows (kernel order) is the oracle's
-    oq, osf, ot = nvfp4.quantize(p["R"][cols], amax=np.max(np.abs(p["R"])))
+    oq, osf, ot, _ = nvfp4.quantize(p["R"][cols], amax=np.max(np.abs(p["R"])))
     inv = np.argsort(perm)                                                # natural row -> kernel row
     assert float(pw.t_w.cpu()[0]) == float(ot)
     np.testing.assert_array_equal(pw.Wq.cpu().numpy()[inv[cols]], nvfp4.pack(oq))
