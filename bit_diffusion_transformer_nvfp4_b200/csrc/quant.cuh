@@ -169,16 +169,20 @@ struct QuantTile {
   static constexpr int kBytes = kQRows * kQChunk * static_cast<int>(sizeof(SrcT));
   static constexpr int kBoxes = sizeof(SrcT) / 2;
   static constexpr int kStages = sizeof(SrcT) == 2 ? 9 : 6;
+  // The producer refills kGroup ring slots at once, so that the loads of
+  // adjacent chunks of the same rows reach DRAM together.
+  static constexpr int kGroup = 3;
   static constexpr int kL1Bytes = 32 * kQChunk * 2;  // L1t tile, 32 x 64 bf16 (4 KB)
   static constexpr int kL1Off = kBytes;
   static constexpr int kInvSOff = kBytes + (sizeof(SrcT) == 2 ? kL1Bytes : 0);  // 64 fp32 of inv_s
   static constexpr int kStageBytes = (kInvSOff + kQChunk * 4 + 1023) / 1024 * 1024;
-  // ring, then per compute warp two 1 KB staging buffers for its codes (32
-  // rows x 32 bytes, written out by TMA), barriers + scalars (512 B), 1 KB
+  // ring, then per compute warp kCodeBufs 1 KB staging buffers for its codes
+  // (32 rows x 32 bytes, written out by TMA), barriers + scalars (512 B), 1 KB
   // alignment slack
   static constexpr int kCodeBuf = 32 * 32;
+  static constexpr int kCodeBufs = 2;
   static constexpr int kCodeOff = kStageBytes * kStages;
-  static constexpr int kBarOff = kCodeOff + kQComputeWarps * 2 * kCodeBuf;
+  static constexpr int kBarOff = kCodeOff + kQComputeWarps * kCodeBufs * kCodeBuf;
   static constexpr int kSmem = kBarOff + 512 + 1024;
   // full/empty/mma_done per stage, acc_full/acc_empty per accumulator, drain;
   // then the TMEM address, abort flag, per-warp maxima and the last-slice flag
@@ -394,6 +398,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       tma_prefetch_desc(&tm_x);
       if (lr) tma_prefetch_desc(&tm_l1);
       const uint32_t inv_bytes = p.inv_s != nullptr ? kQChunk * 4 : 0;
+      int total = 0;  // this CTA's chunks, over all of its items
+      for (int w = blockIdx.x; w < n_items; w += gridDim.x) total += item_chunks(w);
       int c = 0;  // this CTA's chunks, in order
       bool ok = true;
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
@@ -402,13 +408,16 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
         const int n = item_chunks(w);
         for (int i = 0; i < n; ++i, ++c) {
           const int s = c % S;
-          if (c >= S) {
-            const uint32_t ph = ((c / S) - 1) & 1;  // the fill of chunk c - S
-            if (!mbar_wait(smem_u32(&empty[s]), ph, abort_flag, p.status) ||
-                (lr && !mbar_wait(smem_u32(&mma_done[s]), ph, abort_flag, p.status))) {
-              ok = false;
-              break;
+          if (c % Tile::kGroup == 0) {
+            // a new group of chunks: wait until all of its slots are free, so
+            // that its loads go out back to back
+            const int c_end = min(c + Tile::kGroup, total);
+            for (int j = max(c, S); j < c_end && ok; ++j) {
+              const uint32_t ph = ((j / S) - 1) & 1;  // the fill of chunk j - S
+              ok = mbar_wait(smem_u32(&empty[j % S]), ph, abort_flag, p.status) &&
+                   (!lr || mbar_wait(smem_u32(&mma_done[j % S]), ph, abort_flag, p.status));
             }
+            if (!ok) break;
           }
           const uint32_t bar = smem_u32(&full[s]);
           uint8_t* dst = smem + s * Tile::kStageBytes;
@@ -508,8 +517,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
     // ------------------------------------------------------- quantise rows
     const bool has_inv = p.inv_s != nullptr;
     if (lane == 0) tma_prefetch_desc(&tm_q);
-    // this warp's 32 rows of codes go out through two staging buffers
-    uint8_t* code_stage = smem + Tile::kCodeOff + warp * 2 * Tile::kCodeBuf;
+    // this warp's 32 rows of codes go out through kCodeBufs staging buffers
+    uint8_t* code_stage = smem + Tile::kCodeOff + warp * Tile::kCodeBufs * Tile::kCodeBuf;
     int n_stored = 0;
     const int grp = warp >> 2;
     const int row_in_tile = tid & (kQRows - 1);
@@ -566,12 +575,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
       // codes: row ``lane`` of the warp's 32 rows, 32 bytes, into a staging
-      // buffer the TMA store of two chunks ago has finished reading; lanes
-      // with bit 2 set store their halves in the other order (no bank
-      // conflicts); the TMA store drops rows >= M
-      uint8_t* cb = code_stage + (n_stored & 1) * Tile::kCodeBuf;
-      if (n_stored >= 2) {
-        if (lane == 0) bulk_wait_group_read<1>();
+      // buffer whose last TMA store (kCodeBufs chunks of this warp ago) has
+      // finished reading it; lanes with bit 2 set store their halves in the
+      // other order (no bank conflicts); the TMA store drops rows >= M
+      uint8_t* cb = code_stage + (n_stored % Tile::kCodeBufs) * Tile::kCodeBuf;
+      if (n_stored >= Tile::kCodeBufs) {
+        if (lane == 0) bulk_wait_group_read<Tile::kCodeBufs - 1>();
         __syncwarp();
       }
       const int first = (lane >> 2) & 1;
