@@ -182,7 +182,9 @@ struct QuantTile {
   static constexpr int kCodeBuf = 32 * 32;
   static constexpr int kCodeBufs = 2;
   static constexpr int kCodeOff = kStageBytes * kStages;
-  static constexpr int kBarOff = kCodeOff + kQComputeWarps * kCodeBufs * kCodeBuf;
+  // the code multiplier 1/(dec(e) t) of every scale code e (256 fp32)
+  static constexpr int kRqOff = kCodeOff + kQComputeWarps * kCodeBufs * kCodeBuf;
+  static constexpr int kBarOff = kRqOff + 256 * 4;
   static constexpr int kSmem = kBarOff + 512 + 1024;
   // full/empty/mma_done per stage, acc_full/acc_empty per accumulator, drain;
   // then the TMEM address, abort flag, per-warp maxima and the last-slice flag
@@ -391,6 +393,16 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
   const float rt = __frcp_rn(t);
   if (blockIdx.x == 0 && tid == 0) *p.t_out = t;
   const uint32_t tmem = lr ? *tmem_slot : 0u;
+  // The code multiplier 1/(dec(e) t) of every scale code a block can get
+  // (1..126: non-negative, saturated at 448); code 0 leaves the block's codes
+  // +0 and never uses its entry.  The same correctly rounded values the
+  // per-block computation gives, looked up instead of computed.
+  float* rq_tab = reinterpret_cast<float*>(smem + Tile::kRqOff);
+  if (tid < 256)
+    rq_tab[tid] = (tid >= 1 && tid <= 126)
+                      ? __frcp_rn(__fmul_rn(e4m3x2_to_f32(static_cast<uint32_t>(tid)).y, t))
+                      : 0.0f;
+  __syncthreads();
 
   if (warp == kQProducerWarp) {
     // ------------------------------------------------------- TMA producer
@@ -554,17 +566,15 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const uint32_t e = (e2 >> (8 * q)) & 0xFFu;
-          cw[4 * h + 2 * q] = cw[4 * h + 2 * q + 1] = 0u;
-          if (e != 0u) {  // a zero scale leaves the block's codes +0
-            const float rq = __frcp_rn(__fmul_rn(e4m3x2_to_f32(e).y, t));  // 1/(dec(e) t)
+          const float rq = rq_tab[e];  // 1/(dec(e) t)
 #pragma unroll
-            for (int uu = 0; uu < 2; ++uu) {
-              float v[8];
+          for (int uu = 0; uu < 2; ++uu) {
+            float v[8];
 #pragma unroll
-              for (int jj = 0; jj < 8; jj += 2)
-                mul2_rn(v[jj], v[jj + 1], x[16 * q + 8 * uu + jj], x[16 * q + 8 * uu + jj + 1], rq, rq);
-              cw[4 * h + 2 * q + uu] = cvt_e2m1x8(v);
-            }
+            for (int jj = 0; jj < 8; jj += 2)
+              mul2_rn(v[jj], v[jj + 1], x[16 * q + 8 * uu + jj], x[16 * q + 8 * uu + jj + 1], rq, rq);
+            // a zero scale leaves the block's codes +0 (masked, not branched)
+            cw[4 * h + 2 * q + uu] = e != 0u ? cvt_e2m1x8(v) : 0u;
           }
         }
       }
