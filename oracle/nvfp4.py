@@ -164,14 +164,20 @@ def tensor_scale(amax: np.float32) -> np.float32:
     return t
 
 
-def quantize(xs: np.ndarray, amax=None):
+def quantize(xs: np.ndarray, amax=None, t=None):
     """Quantise an already-smoothed fp32 matrix [rows, K] to NVFP4.
 
     ``amax`` is the tensor's absolute maximum; when the rows given are a
     subset of a larger tensor, pass the whole tensor's maximum (once the
     tensor scale is fixed, every row is quantised independently of the
-    others).  Returns ``(codes u8 [rows, K], sf u8 [rows, K/16], t f32,
-    amax f32)``; codes are unpacked (one per byte, see ``pack``).
+    others).  ``t``, if given, is the tensor scale itself (a static or
+    previous-step scale, the calibrated alternative that "SVDQuant Guide:
+    4-Bit DiT Acceleration & Outlier Absorption", "1. Timestep-Aware Outlier
+    Calibration" describes) and replaces ``tensor_scale(amax)``; the block
+    scales and codes follow from it by the same steps, saturating where the
+    data exceed what it can express.  Returns ``(codes u8 [rows, K],
+    sf u8 [rows, K/16], t f32, amax f32)``; codes are unpacked (one per byte,
+    see ``pack``).
     """
     xs = np.asarray(xs, dtype=np.float32)
     rows, K = xs.shape
@@ -180,7 +186,12 @@ def quantize(xs: np.ndarray, amax=None):
     if amax is None:
         amax = F32(np.max(np.abs(xs))) if xs.size else F32(0.0)
     amax = F32(amax)
-    t = tensor_scale(amax)
+    if t is None:
+        t = tensor_scale(amax)
+    else:
+        t = F32(t)
+        if not (t >= F32(2.0 ** -126)) or not np.isfinite(t):
+            raise ValueError("a given tensor scale must be a normal positive fp32 number")
     rt = F32(F32(1.0) / t)
     blocks = xs.reshape(rows, K // BLOCK, BLOCK)
     bmax = np.max(np.abs(blocks), axis=2).astype(np.float32)          # b

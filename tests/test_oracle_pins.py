@@ -413,3 +413,37 @@ def test_swiglu_split_by_hand():
     # gate and up are not interchangeable
     _, h2 = swiglu.split_fused(y[:, [0, 1, 4, 5, 2, 3]], 2, 2)
     assert not np.allclose(h, h2)
+
+
+# ---------------------------------------------------------------- given tensor scale
+
+def test_given_tensor_scale_matches_the_measured_one():
+    g = rng(31)
+    x = bf16_round(g.standard_normal((40, 128)).astype(np.float32) * 3.0)
+    a = np.float32(np.max(np.abs(x)))
+    c1, s1, t1, _ = nvfp4.quantize(x, amax=a)
+    c2, s2, t2, _ = nvfp4.quantize(x, t=nvfp4.tensor_scale(a))
+    assert t1 == t2
+    np.testing.assert_array_equal(c1, c2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_given_tensor_scale_by_hand():
+    # one block [6, -3, 0.5, 0, ...]: with t = 1 its scale is E4M3(6 / 6) =
+    # 1.0 = 0x38 and the codes are the values themselves (6 -> 0x7, -3 -> 0xD,
+    # 0.5 -> 0x1); with t = 2 the scale is E4M3(6 * 0.5 / 6) = 0.5 = 0x30 and
+    # the codes again the values (x / (0.5 * 2)); with t = 1/128 the block
+    # needs 6 * 128 / 6 = 128 -> 0x70 (1.0 * 2^7)
+    x = np.zeros((1, 16), np.float32)
+    x[0, :3] = [6.0, -3.0, 0.5]
+    for t, sbyte in [(1.0, 0x38), (2.0, 0x30), (1.0 / 128, 0x70)]:
+        c, sf, tt, _ = nvfp4.quantize(x, t=t)
+        assert float(tt) == t and sf[0, 0] == sbyte, (t, hex(sf[0, 0]))
+        assert list(c[0, :4]) == [0x7, 0xD, 0x1, 0x0]
+    # a scale too small for the data saturates the block scale at 448 and the
+    # codes at 6: t = 1/1024 asks for 6 * 1024 / 6 = 1024 > 448
+    c, sf, _, _ = nvfp4.quantize(x, t=1.0 / 1024)
+    assert sf[0, 0] == 0x7E
+    assert c[0, 0] == 0x7
+    with pytest.raises(ValueError):
+        nvfp4.quantize(x, t=0.0)
