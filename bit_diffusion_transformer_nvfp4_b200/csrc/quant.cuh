@@ -155,8 +155,8 @@ struct QuantParams {
   float* u_part;           // [splits][row_blocks*128][32] fp32 partial U
   __nv_bfloat16* u_out;    // [M, 64] hi|lo
   int* tickets;            // [row_blocks]
-  int chunks_per_split;
-  int splits;
+  int chunks_per_split;     // single-pass kernel: K slice of each CTA
+  int splits;               // single-pass kernel: K slices per row block
   int row_blocks;
   int has_lr;
   int r;                   // low-rank rank (16 or 32) when has_lr
@@ -253,7 +253,7 @@ __device__ __forceinline__ float tensor_scale_from(float amax) {
 // bf16: hi in columns [0, r), lo in [r, 2r); columns in groups of 16, two
 // slices' loads in flight).
 __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, int64_t rows_pad, int64_t prow,
-                                                 int64_t row) {
+                                                 int64_t row, int n_parts) {
   __threadfence();
   const float ra = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
   __nv_bfloat16* urow = p.u_out + row * 2 * p.r;
@@ -262,11 +262,11 @@ __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, 
     float acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-    for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
+    for (int sp0 = 0; sp0 < n_parts; sp0 += 2) {
       float4 w[2][4];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        if (sp0 + q < p.splits) {
+        if (sp0 + q < n_parts) {
           const float4* src = reinterpret_cast<const float4*>(
               p.u_part + (static_cast<int64_t>(sp0 + q) * rows_pad + prow) * 32 + 16 * hh);
 #pragma unroll
@@ -275,7 +275,7 @@ __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, 
       }
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        if (sp0 + q < p.splits) {
+        if (sp0 + q < n_parts) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             acc[4 * j] = __fadd_rn(acc[4 * j], w[q][j].x);
@@ -350,12 +350,31 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int chunks = static_cast<int>(p.K / kQChunk);
-  const int n_items = p.row_blocks * p.splits;
   const bool lr = p.has_lr != 0;
   grid_launch_dependents();
 
-  // Work item w: row block w / splits, chunks [split * cps, ...) of its K.
-  auto item_chunks = [&](int w) { return min(p.chunks_per_split, chunks - (w % p.splits) * p.chunks_per_split); };
+  // The (row block, chunk) sequence of the whole activation, row block by
+  // row block, is cut into gridDim.x equal contiguous ranges, one per CTA.
+  // A CTA's work items are the pieces of its range that lie in one row block
+  // (rarely more than two); a row block is covered by the pieces of up to
+  // ceil(gridDim / row_blocks) + 1 consecutive CTAs, whose partial U are
+  // summed in CTA order.
+  const int64_t total_chunks = static_cast<int64_t>(p.row_blocks) * chunks;
+  const int64_t g_begin = static_cast<int64_t>(blockIdx.x) * total_chunks / gridDim.x;
+  const int64_t g_end = static_cast<int64_t>(blockIdx.x + 1) * total_chunks / gridDim.x;
+  auto cta_of = [&](int64_t g) {  // the CTA whose range holds chunk g
+    return static_cast<int>(((g + 1) * gridDim.x - 1) / total_chunks);
+  };
+  struct Piece {
+    int rb, kc0, n;
+  };
+  auto piece_at = [&](int64_t g) {  // the item of this CTA that starts at chunk g
+    Piece pc;
+    pc.rb = static_cast<int>(g / chunks);
+    pc.kc0 = static_cast<int>(g - static_cast<int64_t>(pc.rb) * chunks);
+    pc.n = static_cast<int>(min(g_end, static_cast<int64_t>(pc.rb + 1) * chunks) - g);
+    return pc;
+  };
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -410,14 +429,14 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       tma_prefetch_desc(&tm_x);
       if (lr) tma_prefetch_desc(&tm_l1);
       const uint32_t inv_bytes = p.inv_s != nullptr ? kQChunk * 4 : 0;
-      int total = 0;  // this CTA's chunks, over all of its items
-      for (int w = blockIdx.x; w < n_items; w += gridDim.x) total += item_chunks(w);
+      const int total = static_cast<int>(g_end - g_begin);  // this CTA's chunks
       int c = 0;  // this CTA's chunks, in order
       bool ok = true;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
-        const int rb = w / p.splits;
-        const int kc0 = (w % p.splits) * p.chunks_per_split;
-        const int n = item_chunks(w);
+      for (int64_t g = g_begin; g < g_end && ok; g += piece_at(g).n) {
+        const Piece pc = piece_at(g);
+        const int rb = pc.rb;
+        const int kc0 = pc.kc0;
+        const int n = pc.n;
         for (int i = 0; i < n; ++i, ++c) {
           const int s = c % S;
           if (c % Tile::kGroup == 0) {
@@ -454,12 +473,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
     if (lr && lane == 0) {
       int c = 0, j = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++j) {
+      for (int64_t g = g_begin; g < g_end && ok; g += piece_at(g).n, ++j) {
         const int a = j % kQAcc;
         if (j >= kQAcc && !mbar_wait(smem_u32(&acc_empty[a]), ((j / kQAcc) - 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d = tmem + 32u * a;
-        const int n = item_chunks(w);
+        const int n = piece_at(g).n;
         for (int i = 0; i < n; ++i, ++c) {
           const int s = c % S;
           if (!mbar_wait(smem_u32(&full[s]), (c / S) & 1, abort_flag, p.status)) {
@@ -490,10 +509,13 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       const int ut = (warp - kQUWarp0) * 32 + lane;
       const int64_t rows_pad = static_cast<int64_t>(p.row_blocks) * kQRows;
       int j = 0;
-      for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++j) {
+      for (int64_t g = g_begin; g < g_end; g += piece_at(g).n, ++j) {
         const int a = j % kQAcc;
-        const int rb = w / p.splits;
-        const int split = w % p.splits;
+        const int rb = piece_at(g).rb;
+        // this piece's place among the row block's pieces, and their number
+        const int b0 = cta_of(static_cast<int64_t>(rb) * chunks);
+        const int split = static_cast<int>(blockIdx.x) - b0;
+        const int n_parts = cta_of(static_cast<int64_t>(rb + 1) * chunks - 1) - b0 + 1;
         if (!mbar_wait(smem_u32(&acc_full[a]), (j / kQAcc) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         uint32_t u[32];
@@ -512,7 +534,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
         named_bar_sync(2, 128);  // the four U warps' partial rows are out
         if (ut == 0) {
           const int ticket = atomicAdd(&p.tickets[rb], 1);
-          const bool last = ticket == p.splits - 1;
+          const bool last = ticket == n_parts - 1;
           if (last) p.tickets[rb] = 0;  // every slice has taken its ticket
           *last_flag = last ? 1 : 0;
         }
@@ -521,7 +543,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
           // this was the row block's last slice: sum every slice's partial
           // for row ut of the block, in slice order
           const int64_t frow = static_cast<int64_t>(rb) * kQRows + ut;
-          finalize_lowrank(p, t, rows_pad, frow, frow);
+          finalize_lowrank(p, t, rows_pad, frow, frow, n_parts);
         }
       }
     }
@@ -534,18 +556,11 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
     int n_stored = 0;
     const int grp = warp >> 2;
     const int row_in_tile = tid & (kQRows - 1);
-    int w = blockIdx.x;   // the item that holds chunk c
-    int item_c0 = 0;      // its first chunk (this CTA's count)
-    int item_n = w < n_items ? item_chunks(w) : 0;
-    for (int c = grp; w < n_items; c += kQGroups) {
-      while (w < n_items && c >= item_c0 + item_n) {
-        item_c0 += item_n;
-        w += gridDim.x;
-        item_n = w < n_items ? item_chunks(w) : 0;
-      }
-      if (w >= n_items) break;
-      const int rb = w / p.splits;
-      const int kc = (w % p.splits) * p.chunks_per_split + (c - item_c0);
+    const int total = static_cast<int>(g_end - g_begin);
+    for (int c = grp; c < total; c += kQGroups) {
+      const int64_t g = g_begin + c;  // chunk c of this CTA in the whole sequence
+      const int rb = static_cast<int>(g / chunks);
+      const int kc = static_cast<int>(g - static_cast<int64_t>(rb) * chunks);
       const int s = c % S;
       if (!mbar_wait(smem_u32(&full[s]), (c / S) & 1, abort_flag, p.status)) break;
       const uint8_t* tile = smem + s * Tile::kStageBytes;

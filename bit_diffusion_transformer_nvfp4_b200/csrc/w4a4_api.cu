@@ -130,6 +130,7 @@ bool encode_sf(CUtensorMap* m, const void* ptr, int64_t rows, int64_t K, uint32_
 
 struct QuantPlan {
   int64_t row_blocks = 0;
+  int64_t grid = 0;  // CTAs of the streaming pass
   int chunks = 0, splits = 0, chunks_per_split = 0;
   int upart_slices = 0;  // K slices the low-rank partial buffer holds
   size_t off_partials = 0, off_tickets = 0, off_barrier = 0, off_upart = 0, bytes = 0;
@@ -169,12 +170,16 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
   QuantPlan q;
   q.row_blocks = ceil_div(M, kQRows);
   q.chunks = static_cast<int>(K / kQChunk);
-  // Streaming pass: persistent CTAs take the (row block, K slice) items in
-  // turn; pick the slice count whose busiest CTA streams the fewest chunks,
-  // charging four chunks per slice for the partial U it adds to a row block's
-  // sum (ties: fewer slices).
-  q.splits = 1;
-  q.chunks_per_split = q.chunks;
+  // Streaming pass: CTA b of G takes chunks [b T / G, (b + 1) T / G) of the
+  // (row block, chunk) sequence (T chunks in all).  With G = row_blocks x
+  // splits every CTA gets one K slice of one row block; with G = kPlanSms
+  // the ranges are as even as they can be and cross row blocks.  Aligned
+  // slices: pick the slice count whose busiest CTA streams the fewest chunks,
+  // charging four chunks per slice for the partial U it adds to a row
+  // block's sum (ties: fewer slices); even ranges when the aligned plan
+  // would leave SMs idle by more than that charge.
+  const int64_t total = q.row_blocks * q.chunks;
+  int splits = 1;
   int64_t best = -1;
   for (int sp = 1; sp <= kQMaxSplits && sp <= q.chunks; ++sp) {
     const int cps = static_cast<int>(ceil_div(q.chunks, sp));
@@ -183,11 +188,26 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
     const int64_t busiest = ceil_div(q.row_blocks * spl, kPlanSms) * cps + 4 * spl;
     if (best < 0 || busiest < best) {
       best = busiest;
-      q.splits = spl;
-      q.chunks_per_split = cps;
+      splits = spl;
     }
   }
-  const int slices_max = std::max(q.splits, fused_splits(q.row_blocks, q.chunks, kPlanSms));
+  const int64_t even_grid = std::min<int64_t>(total, kPlanSms);
+  const int64_t even_busiest = ceil_div(total, even_grid) + 4 * (ceil_div(even_grid, q.row_blocks) + 1);
+  // (measured: even ranges gain on 16896 x 24576, 8 %, and lose 2 % where
+  // they win by less than a few percent on paper, e.g. 16896 x 6144)
+  const bool aligned = q.row_blocks * splits <= kPlanSms && best <= even_busiest + even_busiest / 32;
+  q.grid = aligned ? q.row_blocks * splits : even_grid;
+  // partial U per row block: one per CTA whose range touches it
+  q.splits = static_cast<int>(std::min<int64_t>(q.chunks, aligned ? splits : ceil_div(q.grid, q.row_blocks) + 1));
+  q.chunks_per_split = q.chunks;
+  // the single-pass path has its own K slices (only when its tile set fits
+  // on the device at once: the condition launch_quant_fused checks)
+  int fused = 1;
+  if (q.row_blocks <= kPlanSms) {
+    const int sp = fused_splits(q.row_blocks, q.chunks, kPlanSms);
+    if (ceil_div(q.chunks, sp) <= kFusedMaxChunks && q.row_blocks * sp <= kPlanSms) fused = sp;
+  }
+  const int slices_max = std::max(q.splits, fused);
   // Fixed layout, the same for every M, K and r (so that one workspace
   // serves any sequence of calls): amax partial maxima; the single-pass
   // grid barrier (launch generation, counters and maximum words per
@@ -349,15 +369,16 @@ int launch_quant(const SrcT* X, int64_t M, int64_t K, int64_t ld, const float* i
   p.u_part = upart;
   p.u_out = static_cast<__nv_bfloat16*>(U);
   p.tickets = tickets;
-  p.chunks_per_split = plan.chunks_per_split;
-  p.splits = plan.splits;
+  p.chunks_per_split = plan.chunks;  // (the streaming kernel takes equal ranges, not K slices)
+  p.splits = 1;
   p.row_blocks = static_cast<int>(plan.row_blocks);
   p.has_lr = r > 0 ? 1 : 0;
   p.r = r;
   p.status = dev->status_ptr;
-  // persistent: one CTA per SM walks the (row block, K slice) work items
-  const int64_t items = plan.row_blocks * plan.splits;
-  const int64_t grid2 = items < dev->num_sms ? items : dev->num_sms;
+  // one CTA per SM at most, each taking its share of the (row block, chunk)
+  // sequence (the plan's grid, or fewer CTAs on a smaller device: then each
+  // row block is touched by no more pieces than the workspace holds)
+  const int64_t grid2 = std::min<int64_t>(plan.grid, dev->num_sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid2), 1, 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);

@@ -292,8 +292,8 @@ int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K,
  *
  * - Sizes whose scratch need, nvfp4_quant_workspace_bytes(M, K, r), exceeds
  *   W4A4_NOALLOC_SCRATCH_BYTES are rejected with W4A4_ERR_SCRATCH_LIMIT
- *   before anything is enqueued (with r = 32 this admits roughly M up to
- *   100k tokens).
+ *   before anything is enqueued (with r = 32 this admits M up to about
+ *   65,000 rows at any K; r = 0 needs only the fixed header).
  * - Every call looks up the device address of the array on the current
  *   device (cudaGetSymbolAddress, with that device current); the first call
  *   for that address zeroes the array on the call's stream, so make the first
