@@ -22,7 +22,7 @@ __all__ = [
     "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
     "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor", "w4a4_set_wait_bound",
     "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
-    "gemm_swiglu",
+    "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,6 +49,9 @@ _SIG = {
                                        _c.c_int, _P, _I64, _P, _P, _P]),
     "w4a4_gemm_swiglu": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _I64, _P, _I64,
                                     _P, _I64, _P, _P, _P]),
+    "w4a4_gemm_quantize_next": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P,
+                                           _c.c_int, _I64, _P, _I64, _P, _I64, _P, _P, _P, _I64, _P, _I64, _I64,
+                                           _P, _P]),
     "w4a4_linear": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _c.c_int, _P, _c.c_int, _P,
                                _P, _c.c_size_t, _P]),
     "nvfp4_quantize_act_noalloc": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P, _P]),
@@ -159,6 +162,15 @@ def w4a4_gemm_swiglu(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_pla
     _check("w4a4_gemm_swiglu", lib().w4a4_gemm_swiglu(
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s), _ptr(next_amax), _stream(stream)))
+
+
+def w4a4_gemm_quantize_next(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, n_plain, Y, ldy, H,
+                            ldh, next_inv_s, next_t, next_q, next_ldq, next_sf, next_K, next_col, next_amax,
+                            stream=None):
+    _check("w4a4_gemm_quantize_next", lib().w4a4_gemm_quantize_next(
+        _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
+        _ptr(bias), epilogue, n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s), _ptr(next_t), _ptr(next_q),
+        next_ldq, _ptr(next_sf), next_K, next_col, _ptr(next_amax), _stream(stream)))
 
 
 def w4a4_linear(X, M, N, K, Wq, Wsf, t_w, inv_s, L1t, L2t, r, bias, epilogue, Y, workspace, stream=None):
@@ -308,6 +320,37 @@ def gemm_swiglu(qa: QuantizedActivation, w: PackedWeight, n_plain: int, Y=None, 
     w4a4_gemm_swiglu(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias, n_plain,
                      Y, Y.stride(0) if Y is not None else 0, H, H.stride(0), next_inv_s, next_amax, stream)
     return Y, H
+
+
+def gemm_quantize_next(qa: QuantizedActivation, w: PackedWeight, next_t, next_inv_s=None, epilogue: int = EPI_NONE,
+                       n_plain=None, store_outputs: bool = True, next_K=None, next_col: int = 0, next_q=None,
+                       next_sf=None, next_amax=None, stream=None):
+    """The GEMM whose epilogue also writes the next layer's NVFP4 codes and
+    scale bytes of its final outputs (Y, or H with ``n_plain`` < N) under
+    the given tensor scale ``next_t``.  Returns (Y, H, next_q, next_sf);
+    Y / H are None when not stored."""
+    dev = qa.Xq.device
+    n_plain = w.N if n_plain is None else n_plain
+    n_out = w.N if n_plain == w.N else (w.N - n_plain) // 2
+    next_K = n_out if next_K is None else next_K
+    Y = H = None
+    if n_plain == w.N:
+        if store_outputs:
+            Y = torch.empty(qa.M, w.N, dtype=torch.bfloat16, device=dev)
+    else:
+        if n_plain:
+            Y = torch.empty(qa.M, n_plain, dtype=torch.bfloat16, device=dev)
+        if store_outputs:
+            H = torch.empty(qa.M, n_out, dtype=torch.bfloat16, device=dev)
+    if next_q is None:
+        next_q = torch.zeros(qa.M, next_K // 2, dtype=torch.uint8, device=dev)
+    if next_sf is None:
+        next_sf = torch.zeros(nvfp4_sf_bytes(qa.M, next_K), dtype=torch.uint8, device=dev)
+    w4a4_gemm_quantize_next(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias,
+                            epilogue, n_plain, Y, 0 if Y is None else Y.stride(0), H, 0 if H is None else H.stride(0),
+                            next_inv_s, next_t, next_q, next_q.stride(0), next_sf, next_K, next_col, next_amax,
+                            stream)
+    return Y, H, next_q, next_sf
 
 
 def linear(X: torch.Tensor, w: PackedWeight, epilogue: int = EPI_NONE, Y=None, workspace=None, stream=None):

@@ -63,6 +63,18 @@ struct GemmParams {
   int n_plain;
   __nv_bfloat16* H;
   int64_t ldh;
+  // Quantise-into-epilogue (CTA-pair kernel only): the final outputs (Y, or
+  // H in SwiGLU mode) are also written as the next layer's NVFP4 codes and
+  // block scales under the given tensor scale *t_next, smoothed by
+  // next_inv_s: output column c is column q_col0 + c of the next layer's
+  // [M, next_K] activation (codes q_next [M, ldq bytes], SF atoms sf_next).
+  // q_next == nullptr: off.  Y / H == nullptr: the bf16 values are not stored.
+  uint8_t* q_next;
+  uint8_t* sf_next;
+  const float* t_next;
+  int64_t ldq;
+  int next_K;
+  int q_col0;
 };
 
 // Shared-memory descriptors of the low-rank pass, K step k (16 columns) of

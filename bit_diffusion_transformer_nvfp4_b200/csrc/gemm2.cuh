@@ -38,8 +38,11 @@
 
 namespace w4a4 {
 
-template <int BN_, int STAGES_, int SF_STAGES_ = 5, int EPI_NBUF_ = 2, bool ALIGN_BASE_ = true>
+template <int BN_, int STAGES_, int SF_STAGES_ = 5, int EPI_NBUF_ = 2, bool ALIGN_BASE_ = true, bool QNEXT_ = false>
 struct Gemm2Cfg {
+  // QNEXT: the epilogue can also quantise its outputs for the next layer
+  // (a separate instantiation, so the plain GEMM keeps its registers)
+  static constexpr bool QNEXT = QNEXT_;
   static constexpr int BN = BN_;                       // tile width (output columns)
   static constexpr int BH = BN / 2;                    // B rows held by each CTA
   static constexpr int STAGES = STAGES_;
@@ -334,6 +337,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int q = warp & 3;               // TMEM lane quarter (rows 32q..32q+31 of this CTA)
     const int h = ew >> 2;                // column half
     const float alpha = __fmul_rn(__ldg(p.t_x), __ldg(p.t_w));
+    // the next layer's tensor scale, when this epilogue quantises for it
+    const float t_next = C::QNEXT && p.q_next != nullptr ? __ldg(p.t_next) : 1.0f;
+    const float rt_next = __frcp_rn(t_next);
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     uint8_t* stage_buf = epi_smem + ew * C::EPI_NBUF * C::EPI_BUF;
     float amax = 0.0f;  // next layer's amax over this thread's stored outputs
@@ -403,6 +409,52 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           amax = fmaxf(amax, fmaxf(v0, v1));
         }
       };
+      // the next layer's NVFP4 codes and scale bytes of the 32 outputs of
+      // this row in ``pk`` (output columns col .. col+31: two 16-blocks),
+      // the same arithmetic as the activation quantiser under the given t
+      auto quant_next = [&](const uint32_t (&pk)[16], int col, int ncols) {
+        const int row = row0 + lane;
+        if (row >= p.M || col >= ncols) return;  // ncols % 32 == 0: the 32 columns are all valid
+        float x[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          x[2 * j] = bf16_lo(pk[j]);
+          x[2 * j + 1] = bf16_hi(pk[j]);
+        }
+        if (p.next_inv_s != nullptr) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 s4 = __ldg(reinterpret_cast<const float4*>(p.next_inv_s + col + j));
+            x[j] = __fmul_rn(x[j], s4.x);
+            x[j + 1] = __fmul_rn(x[j + 1], s4.y);
+            x[j + 2] = __fmul_rn(x[j + 2], s4.z);
+            x[j + 3] = __fmul_rn(x[j + 3], s4.w);
+          }
+        }
+        // two blocks' scale bytes in one conversion; byte 0 = the first block
+        const uint32_t e2 = cvt_e4m3x2(div6(__fmul_rn(absmax16(x + 16), rt_next)),
+                                       div6(__fmul_rn(absmax16(x), rt_next))) & 0xFFFFu;
+        uint32_t cw[4];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const uint32_t e = (e2 >> (8 * q2)) & 0xFFu;
+          const float rq = __frcp_rn(__fmul_rn(e4m3x2_to_f32(e).y, t_next));  // 1/(dec(e) t)
+#pragma unroll
+          for (int uu = 0; uu < 2; ++uu) {
+            float v[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; jj += 2)
+              mul2_rn(v[jj], v[jj + 1], x[16 * q2 + 8 * uu + jj], x[16 * q2 + 8 * uu + jj + 1], rq, rq);
+            cw[2 * q2 + uu] = e != 0u ? cvt_e2m1x8(v) : 0u;  // a zero scale leaves the codes +0
+          }
+        }
+        const int kcol = p.q_col0 + col;  // column in the next layer's activation (multiple of 32)
+        *reinterpret_cast<uint4*>(p.q_next + static_cast<int64_t>(row) * p.ldq + kcol / 2) =
+            make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        const int64_t atom = static_cast<int64_t>(row / 128) * (p.next_K / 64) + kcol / 64;
+        *reinterpret_cast<uint16_t*>(p.sf_next + atom * 512 + (row % 32) * 16 + ((row / 32) % 4) * 4 + (kcol / 16) % 4) =
+            static_cast<uint16_t>(e2);
+      };
       if (n0 < p.n_plain) {
         // ---------------------------------------------------- plain outputs
 #pragma unroll
@@ -434,9 +486,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           stage_row(buf, packed);
           if (p.next_amax != nullptr && p.n_plain == p.N) fold_amax(buf, n, p.N);
+          if constexpr (C::QNEXT) {
+            if (p.q_next != nullptr && p.n_plain == p.N) quant_next(packed, n, p.N);
+          }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
+          if (lane == 0 && p.Y != nullptr) {
             tma_store_2d(&tm_y, smem_u32(buf), n, row0);
             bulk_commit_group();
           }
@@ -486,9 +541,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           stage_row(buf, packed);
           const int hc = hc0 + 32 * c2;
           if (p.next_amax != nullptr) fold_amax(buf, hc, n_h);
+          if constexpr (C::QNEXT) {
+            if (p.q_next != nullptr) quant_next(packed, hc, n_h);
+          }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
+          if (lane == 0 && p.H != nullptr) {
             tma_store_2d(&tm_h, smem_u32(buf), hc, row0);
             bulk_commit_group();
           }

@@ -215,17 +215,6 @@ __device__ __forceinline__ void load8(const uint8_t* tile, int r, int c, float (
   }
 }
 
-// Blackwell packed fp32 multiply: two IEEE round-to-nearest products.
-__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 a, b, d;\n\t"
-      "mov.b64 a, {%2, %3};\n\t"
-      "mov.b64 b, {%4, %5};\n\t"
-      "mul.rn.f32x2 d, a, b;\n\t"
-      "mov.b64 {%0, %1}, d;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // Eight smoothed values of row ``r``, elements 8u..8u+7 of a resident chunk
 // (``inv`` holds the chunk's 64 reciprocal smoothing factors).
 template <typename SrcT>
@@ -303,27 +292,6 @@ __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, 
       dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
     }
   }
-}
-
-// Division by 6 of a non-negative fp32 value, correctly rounded for every
-// input >= 2^-100 (Markstein's correction: one residual step from the
-// rounded reciprocal, P. Markstein, IBM J. Res. Develop. 34(1), 1990; checked
-// against IEEE division on every float from 2^-100 up).  Block maxima below
-// 2^-100 give a zero E4M3 scale either way.
-__device__ __forceinline__ float div6(float x) {
-  const float c = 0.16666667f;  // RN(1/6)
-  const float q0 = __fmul_rn(x, c);
-  return __fmaf_rn(__fmaf_rn(-6.0f, q0, x), c, q0);
-}
-
-// max |v[j]| over 16 values, as a tree (four dependent steps).
-__device__ __forceinline__ float absmax16(const float* v) {
-  float m[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) m[j] = fmaxf(fabsf(v[j]), fabsf(v[j + 8]));
-#pragma unroll
-  for (int j = 0; j < 4; ++j) m[j] = fmaxf(m[j], m[j + 4]);
-  return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
 }
 
 template <typename SrcT>

@@ -42,6 +42,8 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 // slack (the kernel checks that the dynamic shared memory base is 1024-byte
 // aligned and reports W4A4_ERR_DEVICE_LAYOUT otherwise): 226 KB.
 using PairMain = Gemm2Cfg<256, 6, 3, 1, false>;
+// the same configuration whose epilogue can quantise for the next layer
+using PairQNext = Gemm2Cfg<256, 6, 3, 1, false, true>;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -100,6 +102,8 @@ int device_setup(DeviceInfo** out) {
              cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm2_kernel<P192>, cudaFuncAttributeMaxDynamicSharedMemorySize, P192::SMEM) ==
              cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<PairQNext>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  PairQNext::SMEM) == cudaSuccess;
 
   if (!attr_ok) { cudaGetLastError(); return W4A4_ERR_CUDA; }
   d.ok = true;
@@ -180,6 +184,18 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
   // would leave SMs idle by more than that charge.
   const int64_t total = q.row_blocks * q.chunks;
   int splits = 1;
+  if (total == 0) {  // an empty problem: only the fixed part of the layout
+    q.grid = 0;
+    q.splits = 1;
+    q.chunks_per_split = q.chunks;
+    q.off_partials = 0;
+    q.off_barrier = kWsBarrierOff;
+    q.off_tickets = kWsTicketsOff;
+    q.off_upart = kWsUpartOff;
+    q.upart_slices = 1;
+    q.bytes = q.off_upart;
+    return q;
+  }
   int64_t best = -1;
   for (int sp = 1; sp <= kQMaxSplits && sp <= q.chunks; ++sp) {
     const int cps = static_cast<int>(ceil_div(q.chunks, sp));
@@ -442,6 +458,12 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   p.n_plain = static_cast<int>(N);
   p.H = nullptr;
   p.ldh = 0;
+  p.q_next = nullptr;
+  p.sf_next = nullptr;
+  p.t_next = nullptr;
+  p.ldq = 0;
+  p.next_K = 0;
+  p.q_col0 = 0;
   const int64_t tiles = ceil_div(M, C::BM) * ceil_div(N, C::BN);
   const int64_t grid = tiles < dev->num_sms ? tiles : dev->num_sms;
   cudaLaunchConfig_t cfg = {};
@@ -461,13 +483,21 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   return W4A4_OK;
 }
 
+// Quantise-into-epilogue outputs of the CTA-pair kernel (q == nullptr: off).
+struct QuantNext {
+  uint8_t* q = nullptr;
+  uint8_t* sf = nullptr;
+  const float* t = nullptr;
+  int64_t ldq = 0, K = 0, col = 0;
+};
+
 // The CTA-pair kernels: 256 x BN tiles on two SMs (cluster of 2).
 template <class C>
 int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                      int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
                      const void* bias, int epi, void* Y, int64_t ldy, const float* next_inv_s, unsigned* next_amax,
                      cudaStream_t stream, DeviceInfo* dev, int64_t n_plain = -1, void* H = nullptr,
-                     int64_t ldh = 0) {
+                     int64_t ldh = 0, QuantNext qn = QuantNext()) {
   if (n_plain < 0) n_plain = N;
   // SwiGLU outputs fill 32-column boxes from two 32-column accumulator blocks
   if (n_plain < N && (C::BN % 64 != 0 || n_plain % C::BN != 0)) return W4A4_ERR_SHAPE;
@@ -482,17 +512,24 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   if (!encode_sf(&tsb, Wsf, N, K, static_cast<uint32_t>(C::SFB_RB))) return W4A4_ERR_CUDA;
   // plain outputs Y [M, n_plain] and SwiGLU outputs H [M, (N - n_plain) / 2],
   // both written in 32 x 32 boxes
-  if (n_plain > 0 && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(n_plain),
+  if (n_plain > 0 && Y != nullptr && !encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(n_plain),
                                 static_cast<uint64_t>(M), static_cast<uint64_t>(ldy) * 2, 32u, 32u,
                                 CU_TENSOR_MAP_SWIZZLE_64B))
     return W4A4_ERR_CUDA;
-  if (n_plain < N) {
+  if (n_plain < N && H != nullptr) {
     if (!encode_2d(&th, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, H, static_cast<uint64_t>((N - n_plain) / 2),
                    static_cast<uint64_t>(M), static_cast<uint64_t>(ldh) * 2, 32u, 32u, CU_TENSOR_MAP_SWIZZLE_64B))
       return W4A4_ERR_CUDA;
-    if (n_plain == 0) ty = th;  // unused
-  } else {
+    if (n_plain == 0 || Y == nullptr) ty = th;  // unused
+  } else if (n_plain > 0 && Y != nullptr) {
     th = ty;  // unused
+  } else {
+    // neither bf16 output is stored (quantised outputs only): the maps are
+    // never used; give them a valid encoding
+    if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M),
+                   static_cast<uint64_t>(K / 2), 32u, 32u, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return W4A4_ERR_CUDA;
+    th = ty;
   }
   if (r > 0) {
     // U = [hi | lo], rows of 2r bf16; L2t rows of r bf16 (swizzle = row width)
@@ -526,6 +563,12 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   p.n_plain = static_cast<int>(n_plain);
   p.H = static_cast<__nv_bfloat16*>(H);
   p.ldh = ldh;
+  p.q_next = qn.q;
+  p.sf_next = qn.sf;
+  p.t_next = qn.t;
+  p.ldq = qn.ldq;
+  p.next_K = static_cast<int>(qn.K);
+  p.q_col0 = static_cast<int>(qn.col);
   const int64_t tiles = ceil_div(M, 2 * C::BM) * ceil_div(N, C::BN);
   const int64_t max_pairs = dev->num_sms / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -720,6 +763,44 @@ int w4a4_gemm_swiglu(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   return launch_gemm_pair<PairMain>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, W4A4_EPI_NONE, Y, ldy,
                                     next_inv_s, reinterpret_cast<unsigned*>(next_amax),
                                     static_cast<cudaStream_t>(stream), dev, n_plain, H, ldh);
+}
+
+int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M,
+                            int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w,
+                            const void* L2t, int r, const void* bias, int epilogue, int64_t n_plain, void* Y,
+                            int64_t ldy, void* H, int64_t ldh, const float* next_inv_s, const float* next_t,
+                            uint8_t* next_q, int64_t next_ldq, uint8_t* next_sf, int64_t next_K, int64_t next_col,
+                            float* next_amax, void* stream) {
+  if (n_plain < 0 || n_plain > N || n_plain % 256 != 0 && n_plain != N) return W4A4_ERR_SHAPE;
+  const bool swiglu = n_plain < N;
+  if (swiglu && ((N - n_plain) % 32 != 0 || epilogue != W4A4_EPI_NONE)) return W4A4_ERR_SHAPE;
+  const int64_t n_out = swiglu ? (N - n_plain) / 2 : N;  // the outputs quantised for the next layer
+  if (n_out % 32 != 0 || next_K % 64 != 0 || next_col < 0 || next_col % 64 != 0 || next_col + n_out > next_K ||
+      next_ldq < next_K / 2 || next_ldq % 16 != 0 || next_K > (int64_t(1) << 30))
+    return W4A4_ERR_SHAPE;
+  if (swiglu && H != nullptr && (ldh < n_out || ldh % 8 != 0)) return W4A4_ERR_SHAPE;
+  if (n_plain > 0 && Y != nullptr && (ldy < n_plain || ldy % 8 != 0)) return W4A4_ERR_SHAPE;
+  if (swiglu && n_plain > 0 && Y == nullptr) return W4A4_ERR_NULL;  // the plain (unquantised) outputs
+  int st = check_gemm_args(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, next_q, N);
+  if (st != W4A4_OK || M == 0) return st;
+  if (!next_sf || !next_t) return W4A4_ERR_NULL;
+  if (!aligned16(next_sf) || reinterpret_cast<uintptr_t>(next_t) % 4 != 0 || (Y && !aligned16(Y)) ||
+      (H && !aligned16(H)) || (next_inv_s && !aligned16(next_inv_s)) ||
+      reinterpret_cast<uintptr_t>(next_amax) % 4 != 0)
+    return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  QuantNext qn;
+  qn.q = next_q;
+  qn.sf = next_sf;
+  qn.t = next_t;
+  qn.ldq = next_ldq;
+  qn.K = next_K;
+  qn.col = next_col;
+  return launch_gemm_pair<PairQNext>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
+                                     next_inv_s, reinterpret_cast<unsigned*>(next_amax),
+                                     static_cast<cudaStream_t>(stream), dev, n_plain, H, ldh, qn);
 }
 
 int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,

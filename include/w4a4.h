@@ -263,6 +263,51 @@ int w4a4_gemm_swiglu(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
                      float* next_amax, void* stream);
 
 /*
+ * w4a4_gemm_quantize_next -- w4a4_gemm (epilogue NONE or GELU_TANH) or
+ * w4a4_gemm_swiglu (n_plain < N) whose epilogue also quantises its final
+ * outputs for the next layer, so that layer's activation quantiser need not
+ * read them: the fusion the SVDQuant guide's engine section motivates ("SVDQuant
+ * Guide: 4-Bit DiT Acceleration & Outlier Absorption", "3. The Nunchaku Fused
+ * Kernel Engine": no second kernel streaming the same tensor), under a tensor
+ * scale the caller gives (a static calibration, "1. Timestep-Aware Outlier
+ * Calibration", or the previous step's), which is what makes it possible in
+ * one pass: the scale no longer comes from this step's amax.
+ *   The final outputs F are Y (n_plain == N; after bias and the epilogue) or
+ *   H (the SwiGLU outputs).  Column c of F is column next_col + c of the next
+ *   layer's [M, next_K] activation; for every row m and 16-block of F, with
+ *   x~ = fl(bf16(F[m,c]) * next_inv_s[c]) and t = *next_t, the kernel writes
+ *   the scale byte E4M3_rn_satfinite((b * (1/t)) / 6) and the codes
+ *   E2M1_rn_satfinite(x~ * (1 / (dec(e) t))) (+0 for a zero scale) of
+ *   nvfp4_quantize_act -- bit for bit what nvfp4_quantize_act would write for
+ *   these columns of the bf16 outputs if its tensor scale were t.
+ *   next_inv_s  in   fp32 [n_out] (n_out = N, or (N - n_plain) / 2), or NULL for ones
+ *   next_t      in   fp32 device scalar, the next layer's tensor scale (> 0,
+ *                    a normal number); pass it as that layer's t_x
+ *   next_q      out  uint8 codes [M, next_ldq bytes], next_ldq >= next_K / 2,
+ *                    next_ldq % 16 == 0; bytes [next_col / 2, (next_col + n_out) / 2)
+ *                    of each row are written
+ *   next_sf     out  SF atoms of the [M, next_K] activation (nvfp4_sf_bytes(M,
+ *                    next_K) bytes); the scale bytes of those columns for rows
+ *                    < M are written (pad rows are left as they are)
+ *   next_K, next_col  next_K % 64 == 0, next_col % 64 == 0, next_col + n_out <= next_K
+ *   next_amax   as in w4a4_gemm_next_amax (over F), or NULL
+ *   Y / H       as in w4a4_gemm / w4a4_gemm_swiglu; may be NULL to skip
+ *               storing the bf16 values (Y must be given when n_plain is
+ *               between 0 and N: those outputs are not quantised)
+ * The next layer's low-rank input U = F L1 still needs the bf16 F (the
+ * quantiser with the amax given computes it); a next layer without a
+ * low-rank branch needs only next_q, next_sf and next_t.  n_out % 32 == 0.
+ * Launches one CTA-pair GEMM kernel.
+ */
+int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U,
+                            int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,
+                            const float* t_w, const void* L2t, int r, const void* bias, int epilogue,
+                            int64_t n_plain, void* Y, int64_t ldy, void* H, int64_t ldh,
+                            const float* next_inv_s, const float* next_t, uint8_t* next_q,
+                            int64_t next_ldq, uint8_t* next_sf, int64_t next_K, int64_t next_col,
+                            float* next_amax, void* stream);
+
+/*
  * w4a4_linear -- the whole hot path: nvfp4_quantize_act on X (row stride K)
  * into the workspace, then w4a4_gemm into Y (row stride N).
  *   workspace >= w4a4_workspace_bytes(M, N, K, r) bytes of device memory.

@@ -204,3 +204,34 @@ def test_swiglu_argument_checks(so):
     assert f(P, P, P, None, 128, 1024, 512, P, P, P, None, 0, None, 256, P, 256, P + 2, 384, None, None, None) == -3
     assert f(None, None, None, None, 0, 1024, 512, None, None, None, None, 0, None, 256, None, 256, None, 384,
              None, None, None) == 0
+
+
+def test_quantize_next_argument_checks(so):
+    """w4a4_gemm_quantize_next rejects bad column ranges, strides and pointers on the host."""
+    P = 1 << 20
+    f = so.w4a4_gemm_quantize_next
+    #          Xq Xsf t_x U  M    N    K    Wq Wsf t_w L2t  r  bias epi n_plain Y  ldy H  ldh s  t  q  ldq sf nK   col  amax stream
+    ok = dict(n_plain=384, next_K=384, col=0, ldq=192)
+    def call(n_plain=384, next_K=384, col=0, ldq=192, t=P, sf=P, q=P, epi=0, N=384):
+        return f(P, P, P, None, 128, N, 512, P, P, P, None, 0, None, epi, n_plain, P, N, None, 0, None, t, q, ldq,
+                 sf, next_K, col, None, None)
+    if not __import__("torch").cuda.is_available():
+        assert call() == -4                                    # valid: reaches the device check
+    assert call(next_K=320) == -2                              # columns beyond next_K
+    assert call(next_K=448, col=64) == -2                      # 448 % 64 ok, but col + 384 > 448
+    assert call(next_K=512, col=32) == -2                      # column offset not a multiple of 64
+    assert call(ldq=176) == -2                                 # codes row shorter than next_K / 2
+    assert call(t=None) == -1                                  # no tensor scale
+    assert call(q=None) == -1
+    assert call(sf=P + 4) == -3
+    assert call(n_plain=200) == -2                             # SwiGLU split not a multiple of 256
+    assert call(n_plain=0, N=416, next_K=256) == -2            # SwiGLU outputs 208 not a multiple of 32
+    assert call(epi=7) == -8
+
+
+def test_sizes_of_empty_problems(so):
+    """Size queries for M == 0 (an empty batch) return the fixed layout, not a crash."""
+    upart = 5120 + 4 * ((1 << 22) // 128)
+    for r in (0, 16, 32):
+        assert so.nvfp4_quant_workspace_bytes(0, 512, r) == upart
+        assert so.w4a4_workspace_bytes(0, 384, 512, r) >= upart
