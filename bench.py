@@ -616,26 +616,36 @@ def run_table(args):
     def emit(row):
         print(json.dumps(row), flush=True)
 
-    def prepare(case, bias=True):
+    swiglu_split = {(4, "qkv_swiglu_up"): 18432}  # the fused projection: plain QKV, then SwiGLU pairs
+
+    def prepare(case, bias=True, n_plain=None):
         W = dev_bf16(case.w)
         Xc = dev_bf16(case.x_cal)
         b = dev_bf16(case.bias) if (bias and case.bias is not None) else None
+        if n_plain is not None:  # the kernel's row order for the SwiGLU epilogue
+            order = prep.swiglu_row_order(n_plain, (case.N - n_plain) // 2, device=dev)
+            W = W[order].contiguous()
+            b = None if b is None else b[order].contiguous()
         pk = prep.svdquant_prepare(W, Xc, r=case.r, bias=b)
         del W, Xc
         return pk
 
-    def linear_row(cfg, case, pk, X, epi=0):
+    def linear_row(cfg, case, pk, X, epi=0, n_plain=None):
         M, K, N, r = X.shape[0], X.shape[1], pk.N, pk.r
         ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, r), dev)
         qa = w4.quantize_act(X, pk.inv_s, pk.L1t, pk.t_w, workspace=ws)
-        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        Y = torch.empty(M, N if n_plain is None else n_plain, dtype=torch.bfloat16, device=dev)
+        H = None if n_plain is None else torch.empty(M, (N - n_plain) // 2, dtype=torch.bfloat16, device=dev)
 
         def qi():
             w4.nvfp4_quantize_act(X, M, K, X.stride(0), pk.inv_s, pk.L1t, r, pk.t_w, qa.Xq, qa.Xsf, qa.t_x,
                                   qa.U, ws, s)
 
         def g():
-            w4.gemm(qa, pk, epilogue=epi, Y=Y)
+            if n_plain is None:
+                w4.gemm(qa, pk, epilogue=epi, Y=Y)
+            else:
+                w4.gemm_swiglu(qa, pk, n_plain, Y=Y, H=H)
 
         def both():
             qi()
@@ -648,7 +658,7 @@ def run_table(args):
         gfl = gemm_flops(M, K, N, r)
         qbytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * M * 2 * r
         row = {"table": "linear", "config": cfg, "layer": case.name, "M": M, "K": K, "N": N, "r": r,
-               "epilogue": "gelu_tanh" if epi else "none",
+               "epilogue": "swiglu" if n_plain is not None else ("gelu_tanh" if epi else "none"),
                "quant_us": round(tq, 2), "quant_gbs": round(qbytes / (tq * 1e-6) / 1e9, 1),
                "quant_frac_hbm": round(qbytes / (tq * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
                "gemm_us": round(tg, 2), "gemm_tflops": tf(gfl, tg), "gemm_frac_fp4": round(tf(gfl, tg) / fp4_peak, 3),
@@ -657,6 +667,33 @@ def run_table(args):
                "linear_frac_fp4": round(tf(fl, tl) / fp4_peak, 3)}
         emit(row)
         return qa, ws, Y, qi, g
+
+    def quant_next_row(cfg, case, pk, qa, g, epi=0, n_plain=None, next_K=None, next_col=0):
+        """The GEMM whose epilogue also writes the next layer's NVFP4 codes and
+        scale bytes (w4a4_gemm_quantize_next, given tensor scale), with and
+        without storing the bf16 outputs, beside the plain GEMM."""
+        M, N = qa.M, pk.N
+        n_out = N if n_plain is None else (N - n_plain) // 2
+        next_K = n_out if next_K is None else next_K
+        t_next = torch.full((1,), 0.01, device=dev)
+        s_next = torch.ones(n_out, device=dev)
+        nq = torch.empty(M, next_K // 2, dtype=torch.uint8, device=dev)
+        nsf = torch.empty(w4.nvfp4_sf_bytes(M, next_K), dtype=torch.uint8, device=dev)
+        outs = {}
+
+        def gq(store):
+            def f():
+                w4.gemm_quantize_next(qa, pk, t_next, next_inv_s=s_next, epilogue=epi, n_plain=n_plain,
+                                      store_outputs=store, next_K=next_K, next_col=next_col, next_q=nq,
+                                      next_sf=nsf)
+            return f
+        t_plain, t_store, t_codes = med_us([g, gq(True), gq(False)])
+        check()
+        gfl = gemm_flops(M, case.K, N, pk.r)
+        emit({"table": "quantise_into_epilogue", "config": cfg, "layer": case.name, "M": M, "K": case.K, "N": N,
+              "outputs_quantised": n_out, "gemm_us": round(t_plain, 2),
+              "gemm_with_next_codes_us": round(t_store, 2), "gemm_next_codes_only_us": round(t_codes, 2),
+              "gemm_next_codes_only_tflops": tf(gfl, t_codes)})
 
     emit({"table": "peaks", "fp4_peak_tflops": round(fp4_peak, 1), "hbm_gbs": peaks["hbm_gbs"],
           "basis": f"{peak_kind}: bf16 burst x {FP4_OVER_BF16:g}; copy bandwidth", "reps": reps,
@@ -694,14 +731,19 @@ def run_table(args):
             row["graph_error"] = str(exc)[:200]
         emit(row)
 
-    # configs 1, 2, 4: independent linears
+    # configs 1, 2, 4: independent linears (config 4's fused projection with
+    # its SwiGLU epilogue, and quantising its SwiGLU outputs into columns
+    # 6144.. of the output projection's 24576-wide activation)
     for cfg in (1, 2, 4):
         for case in config_cases(cfg):
-            pk = prepare(case)
+            n_plain = swiglu_split.get((cfg, case.name))
+            pk = prepare(case, n_plain=n_plain)
             X = dev_bf16(case.x)
-            qa, ws, Y, qi, g = linear_row(cfg, case, pk, X)
+            qa, ws, Y, qi, g = linear_row(cfg, case, pk, X, n_plain=n_plain)
             if cfg == 1:
                 graph_row(case, pk, X, qa, ws, Y, qi, g)
+            if n_plain is not None:
+                quant_next_row(cfg, case, pk, qa, g, n_plain=n_plain, next_K=24576, next_col=6144)
             del pk, X, qa, ws, Y
             torch.cuda.empty_cache()
 
@@ -710,6 +752,7 @@ def run_table(args):
     pu, pd = prepare(up), prepare(down)
     X = dev_bf16(up.x)
     qa_u, ws_u, H, qi_u, g_u = linear_row(3, up, pu, X, epi=1)
+    quant_next_row(3, up, pu, qa_u, g_u, epi=1)
     M = up.M
     ws_d = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, down.K, down.r), dev)
     qa_d = w4.quantize_act(H, pd.inv_s, pd.L1t, pd.t_w, workspace=ws_d)
