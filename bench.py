@@ -857,6 +857,9 @@ CASES = {
     "gemm_block2048_up": ("w4a4_gemm_swiglu, the 2048px fused QKV+SwiGLU-up projection", 16896, 6144, 55296, 18432),
     "gemm_block2048_up_small": ("w4a4_gemm_swiglu, the 2048px fused projection at 4096 tokens", 4096, 6144, 55296, 18432),
     "gemm_block2048_out": ("w4a4_gemm, the 2048px output projection", 16896, 24576, 6144, None),
+    "gemm_quant_next_block2048_small": ("w4a4_gemm_quantize_next, the 2048px fused projection at 4096 tokens, its "
+                                        "SwiGLU outputs quantised into columns 6144.. of a 24576-wide activation",
+                                        4096, 6144, 55296, 18432),
     "gemm_flux1024_qkv": ("w4a4_gemm, the FLUX-1024px QKV projection (CTA pairs, 256 x 256 tiles)", 4608, 3072, 9216, None),
     "gemm_row_block": ("w4a4_gemm on a single 128-row block (CTA pairs, 256 x 64 tiles)", 128, 3072, 3072, None),
     "gemm_single_cta": ("w4a4_gemm on a single row block with N > 64 SMs (single-CTA 128 x 192 tiles)", 64, 3072, 19200,
@@ -913,7 +916,18 @@ def run_case(args):
             pw = w4.pack_weight(W)
             del W
             L2t = (0.02 * torch.randn(N, r, generator=g, device=dev)).to(torch.bfloat16)
-            if n_plain is None:
+            if args.case.startswith("gemm_quant_next"):
+                Y = torch.empty(M, n_plain, dtype=torch.bfloat16, device=dev)
+                H = torch.empty(M, (N - n_plain) // 2, dtype=torch.bfloat16, device=dev)
+                t_next = torch.full((1,), 0.01, device=dev)
+                nq = torch.empty(M, 24576 // 2, dtype=torch.uint8, device=dev)
+                nsf = torch.empty(w4.nvfp4_sf_bytes(M, 24576), dtype=torch.uint8, device=dev)
+
+                def call():
+                    w4.w4a4_gemm_quantize_next(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, pw.Wq, pw.Wsf, pw.t_w, L2t, r,
+                                               None, 0, n_plain, Y, n_plain, H, H.shape[1], None, t_next, nq,
+                                               nq.stride(0), nsf, 24576, 6144, None, st)
+            elif n_plain is None:
                 Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
 
                 def call():
