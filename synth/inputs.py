@@ -22,7 +22,7 @@ import numpy as np
 
 __all__ = [
     "bf16_bits", "bf16_round", "bits_to_f32", "LinearCase", "make_linear",
-    "CONFIGS", "config_cases", "trajectory_step_activation", "rng",
+    "CONFIGS", "config_cases", "trajectory_step_activation", "rng", "token_positions",
 ]
 
 
@@ -147,6 +147,17 @@ def make_linear(name, M, K, N, r=32, act="normal_outliers", n_out=8, out_scale=1
         bias = bf16_round((bias_std * gw.standard_normal(N, dtype=np.float32)).astype(np.float32))
     return LinearCase(name, M, K, N, r, bf16_round(x), bf16_round(w), bias,
                       bf16_round(xc), alpha, meta)
+
+
+def token_positions(n_text: int, h: int, w: int, batch: int = 1) -> np.ndarray:
+    """Integer positions [batch * (n_text + h * w), 3] of a joint text + image
+    token sequence, per image: the text tokens first, all at (0, 0, 0), then
+    the h x w latent patches in row-major order at (0, row, column).  Pure
+    indices: no draw and no arithmetic of the method."""
+    img = np.stack(np.meshgrid(np.arange(h), np.arange(w), indexing="ij"), axis=-1).reshape(-1, 2)
+    one = np.concatenate([np.zeros((n_text, 3), np.int64),
+                          np.concatenate([np.zeros((h * w, 1), np.int64), img], axis=1)])
+    return np.tile(one, (batch, 1))
 
 
 # --------------------------------------------------------------------------

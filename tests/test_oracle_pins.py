@@ -447,3 +447,73 @@ def test_given_tensor_scale_by_hand():
     assert c[0, 0] == 0x7
     with pytest.raises(ValueError):
         nvfp4.quantize(x, t=0.0)
+
+
+# ---------------------------------------------------------------- rotary embedding
+
+def test_rope_rotation_by_hand():
+    from oracle import rope
+    # one head of 4 features (pairs (0,1) and (2,3)) then two plain columns;
+    # pair 0 turned by a quarter turn, pair 1 by a half turn
+    y = np.array([[1.0, 0.0, 0.0, 1.0, 3.0, 4.0]])
+    tab = rope.table(np.array([[np.pi / 2, np.pi]]))
+    got = rope.rotate(y, tab, n_rope=4, d_head=4)
+    np.testing.assert_allclose(got, [[0.0, 1.0, 0.0, -1.0, 3.0, 4.0]], atol=1e-7)
+    # a sixth of a turn on (2, 0): (2 cos, 2 sin) = (1, sqrt 3); the pairs are
+    # adjacent features, not the two halves of the head
+    got = rope.rotate(np.array([[2.0, 0.0, 0.0, 0.0]]), rope.table(np.array([[np.pi / 3, 0.0]])), 4, 4)
+    np.testing.assert_allclose(got, [[1.0, np.sqrt(3.0), 0.0, 0.0]], atol=1e-7)
+
+
+def test_rope_every_head_uses_the_same_pairs():
+    from oracle import rope
+    g = rng(41)
+    y = g.standard_normal((3, 24))
+    tab = rope.table(g.uniform(-np.pi, np.pi, (3, 4)))
+    got = rope.rotate(y, tab, n_rope=16, d_head=8)
+    for h0 in (0, 8):
+        np.testing.assert_allclose(got[:, h0:h0 + 8], rope.rotate(y[:, h0:h0 + 8], tab, 8, 8), rtol=0, atol=0)
+    np.testing.assert_array_equal(got[:, 16:], y[:, 16:])        # past n_rope: unchanged
+
+
+def test_rope_preserves_pair_norms_and_inverts():
+    from oracle import rope
+    g = rng(42)
+    y = g.standard_normal((5, 32))
+    th = g.uniform(-10, 10, (5, 8))
+    got = rope.rotate(y, rope.table(th), 32, 16)
+    np.testing.assert_allclose(got[:, 0::2] ** 2 + got[:, 1::2] ** 2, y[:, 0::2] ** 2 + y[:, 1::2] ** 2, rtol=1e-6)
+    back = rope.rotate(got, rope.table(-th), 32, 16)
+    np.testing.assert_allclose(back, y, atol=1e-6)
+
+
+def test_rope_angles_closed_form():
+    from oracle import rope
+    # one axis: RoFormer's theta_i = m base^(-2i/d)
+    th = rope.angles(np.array([[0.0], [1.0], [7.0]]), (8,), 10000.0)
+    want = np.power(10000.0, -np.arange(0, 8, 2) / 8.0)
+    np.testing.assert_allclose(th, np.array([0.0, 1.0, 7.0])[:, None] * want[None, :], rtol=1e-15)
+    np.testing.assert_allclose(th[1], [1.0, 0.1, 0.01, 0.001], rtol=1e-12)
+    # two axes: each owns its own run of pairs and its own frequencies
+    th2 = rope.angles(np.array([[2.0, 5.0]]), (4, 8), 100.0)
+    np.testing.assert_allclose(th2[0], [2.0, 2.0 / 10.0, 5.0, 5.0 / np.sqrt(10.0), 5.0 / 10.0, 5.0 / 10.0 ** 1.5],
+                               rtol=1e-12)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    # the property that makes it a position encoding: the score of a rotated
+    # query and key is unchanged when both positions move by the same offset
+    from oracle import rope
+    g = rng(43)
+    q = g.standard_normal((1, 16))
+    k = g.standard_normal((1, 16))
+    dims, base = (4, 6, 6), 10000.0
+
+    def score(pq, pk):
+        tq = rope.table(rope.angles(np.array([pq], np.float64), dims, base))
+        tk = rope.table(rope.angles(np.array([pk], np.float64), dims, base))
+        return float((rope.rotate(q, tq, 16, 16) @ rope.rotate(k, tk, 16, 16).T)[0, 0])
+
+    s0 = score([0, 3, 9], [0, 1, 4])
+    assert abs(score([5, 10, 12], [5, 8, 7]) - s0) < 1e-5
+    assert abs(score([0, 4, 9], [0, 1, 4]) - s0) > 1e-3           # a different offset does change it
