@@ -22,7 +22,7 @@ __all__ = [
     "QuantizedActivation", "PackedWeight", "quantize_act", "pack_weight", "linear", "gemm",
     "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor", "w4a4_set_wait_bound",
     "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
-    "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next",
+    "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next", "w4a4_gemm_rope", "gemm_rope",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,6 +49,8 @@ _SIG = {
                                        _c.c_int, _P, _I64, _P, _P, _P]),
     "w4a4_gemm_swiglu": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _I64, _P, _I64,
                                     _P, _I64, _P, _P, _P]),
+    "w4a4_gemm_rope": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _I64, _I64, _P,
+                                  _I64, _I64, _P, _I64, _P, _I64, _P, _P, _P]),
     "w4a4_gemm_quantize_next": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P,
                                            _c.c_int, _I64, _P, _I64, _P, _I64, _P, _P, _P, _I64, _P, _I64, _I64,
                                            _P, _P]),
@@ -162,6 +164,14 @@ def w4a4_gemm_swiglu(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_pla
     _check("w4a4_gemm_swiglu", lib().w4a4_gemm_swiglu(
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s), _ptr(next_amax), _stream(stream)))
+
+
+def w4a4_gemm_rope(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_rope, d_head, rope, ld_rope, n_plain, Y,
+                   ldy, H, ldh, next_inv_s, next_amax, stream=None):
+    _check("w4a4_gemm_rope", lib().w4a4_gemm_rope(
+        _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
+        _ptr(bias), n_rope, d_head, _ptr(rope), ld_rope, n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s),
+        _ptr(next_amax), _stream(stream)))
 
 
 def w4a4_gemm_quantize_next(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, n_plain, Y, ldy, H,
@@ -319,6 +329,25 @@ def gemm_swiglu(qa: QuantizedActivation, w: PackedWeight, n_plain: int, Y=None, 
         H = torch.empty(qa.M, n_h, dtype=torch.bfloat16, device=dev)
     w4a4_gemm_swiglu(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias, n_plain,
                      Y, Y.stride(0) if Y is not None else 0, H, H.stride(0), next_inv_s, next_amax, stream)
+    return Y, H
+
+
+def gemm_rope(qa: QuantizedActivation, w: PackedWeight, rope, n_rope: int, d_head: int, n_plain=None, Y=None,
+              H=None, stream=None, next_inv_s=None, next_amax=None):
+    """The fused projection with the rotary embedding on its first ``n_rope``
+    outputs (heads of ``d_head`` features; ``rope`` fp32 [M, >= d_head], per
+    token the (cos, sin) of each feature pair, interleaved) and, with
+    ``n_plain`` < N, the SwiGLU epilogue on the rest as in ``gemm_swiglu``.
+    Returns (Y, H); H is None without SwiGLU outputs."""
+    dev = qa.Xq.device
+    n_plain = w.N if n_plain is None else n_plain
+    if Y is None:
+        Y = torch.empty(qa.M, n_plain, dtype=torch.bfloat16, device=dev)
+    if H is None and n_plain < w.N:
+        H = torch.empty(qa.M, (w.N - n_plain) // 2, dtype=torch.bfloat16, device=dev)
+    w4a4_gemm_rope(qa.Xq, qa.Xsf, qa.t_x, qa.U, qa.M, w.N, w.K, w.Wq, w.Wsf, w.t_w, w.L2t, w.r, w.bias, n_rope,
+                   d_head, rope, rope.stride(0), n_plain, Y, Y.stride(0), H, 0 if H is None else H.stride(0),
+                   next_inv_s, next_amax, stream)
     return Y, H
 
 

@@ -75,6 +75,14 @@ struct GemmParams {
   int64_t ldq;
   int next_K;
   int q_col0;
+  // Rotary embedding (CTA-pair kernel, ROPE instantiation): plain outputs
+  // n < n_rope form heads of d_head features; features 2i, 2i+1 of a head
+  // are turned by the angle whose (cos, sin) are rope[m * ld_rope + 2i],
+  // rope[m * ld_rope + 2i + 1] for token m.  n_rope == 0: off.
+  int n_rope;
+  int d_head;
+  const float* rope;
+  int64_t ld_rope;
 };
 
 // Shared-memory descriptors of the low-rank pass, K step k (16 columns) of

@@ -38,11 +38,14 @@
 
 namespace w4a4 {
 
-template <int BN_, int STAGES_, int SF_STAGES_ = 5, int EPI_NBUF_ = 2, bool ALIGN_BASE_ = true, bool QNEXT_ = false>
+template <int BN_, int STAGES_, int SF_STAGES_ = 5, int EPI_NBUF_ = 2, bool ALIGN_BASE_ = true, bool QNEXT_ = false,
+          bool ROPE_ = false>
 struct Gemm2Cfg {
-  // QNEXT: the epilogue can also quantise its outputs for the next layer
-  // (a separate instantiation, so the plain GEMM keeps its registers)
+  // QNEXT: the epilogue can also quantise its outputs for the next layer;
+  // ROPE: it can rotate the leading plain outputs by the rotary embedding
+  // (separate instantiations, so the plain GEMM keeps its registers)
   static constexpr bool QNEXT = QNEXT_;
+  static constexpr bool ROPE = ROPE_;
   static constexpr int BN = BN_;                       // tile width (output columns)
   static constexpr int BH = BN / 2;                    // B rows held by each CTA
   static constexpr int STAGES = STAGES_;
@@ -73,8 +76,10 @@ struct Gemm2Cfg {
   static constexpr int EPI_WARP0 = 8;                  // warps 8-15: epilogue
   static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
   // registers per thread after setmaxnreg: producer / MMA warpgroup, scale
-  // warpgroup, the two epilogue warpgroups (launch: 65536 / THREADS = 128)
-  static constexpr int REGS_CTRL = 64, REGS_SF = 64, REGS_EPI = 176;
+  // warpgroup, the two epilogue warpgroups (launch: 65536 / THREADS = 128);
+  // the rotary epilogue holds the table values beside the accumulator's, so
+  // its instantiation moves 8 registers from each of the first two to them
+  static constexpr int REGS_CTRL = ROPE ? 56 : 64, REGS_SF = ROPE ? 56 : 64, REGS_EPI = ROPE ? 184 : 176;
   static constexpr int HALF = BN / 2;                  // columns per epilogue warp
   static constexpr int EPI_BUF = 32 * 64;              // 32 rows x 32 bf16, one staging buffer
   static constexpr int EPI_NBUF = EPI_NBUF_;           // staging buffers per epilogue warp
@@ -460,10 +465,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < C::HALF / 32; ++c, ++chunk) {
           const int n = n0 + h * C::HALF + 32 * c;
+          // rotary embedding of this block (32 features of one head): the
+          // (cos, sin) of its 16 pairs for this thread's token, 128 bytes of
+          // the token's table row, read eight values per group of outputs
+          // (a whole block's 32 would not fit beside the accumulator values
+          // without spilling); rows past M read the last row (their outputs
+          // are dropped by the store)
+          const bool rot = C::ROPE && n < p.n_rope;  // the same for the whole warp
+          const float4* src = nullptr;
+          if constexpr (C::ROPE)
+            src = reinterpret_cast<const float4*>(p.rope + static_cast<int64_t>(min(row0 + lane, p.M - 1)) * p.ld_rope +
+                                                  n % p.d_head);
           uint8_t* buf = next_buf();
           uint32_t packed[16];
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
+            float cs[8];
+            if constexpr (C::ROPE) {
+              if (rot) {
+                const float4 v0 = __ldg(src + 2 * g), v1 = __ldg(src + 2 * g + 1);
+                cs[0] = v0.x; cs[1] = v0.y; cs[2] = v0.z; cs[3] = v0.w;
+                cs[4] = v1.x; cs[5] = v1.y; cs[6] = v1.z; cs[7] = v1.w;
+              }
+            }
             float b[8];
             if (p.bias != nullptr && n + 8 * g < p.n_plain) {
               const uint4 bw = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8 * g));
@@ -477,9 +501,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             for (int j = 0; j < 8; j += 2) {
               float y0 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j])), b[j]);
               float y1 = __fadd_rn(__fmul_rn(alpha, __uint_as_float(r[32 * c + 8 * g + j + 1])), b[j + 1]);
-              if (p.epi == 1) {
+              if (!C::ROPE && p.epi == 1) {  // (the rotary entry point has no GELU)
                 y0 = gelu_tanh_f32(y0);
                 y1 = gelu_tanh_f32(y1);
+              }
+              if constexpr (C::ROPE) {
+                if (rot) {
+                  // pair (8g + j) / 2 of the block: (y0, y1) turned by its angle
+                  const float co = cs[j], si = cs[j + 1];
+                  const float r0 = __fmaf_rn(y0, co, -__fmul_rn(y1, si));
+                  const float r1 = __fmaf_rn(y0, si, __fmul_rn(y1, co));
+                  y0 = r0;
+                  y1 = r1;
+                }
               }
               packed[4 * g + j / 2] = pack_bf16x2(y0, y1);
             }

@@ -44,6 +44,8 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 using PairMain = Gemm2Cfg<256, 6, 3, 1, false>;
 // the same configuration whose epilogue can quantise for the next layer
 using PairQNext = Gemm2Cfg<256, 6, 3, 1, false, true>;
+// ... and the one whose epilogue can apply the rotary embedding
+using PairRope = Gemm2Cfg<256, 6, 3, 1, false, false, true>;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -104,6 +106,8 @@ int device_setup(DeviceInfo** out) {
              cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(gemm2_kernel<PairQNext>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PairQNext::SMEM) == cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(gemm2_kernel<PairRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  PairRope::SMEM) == cudaSuccess;
 
   if (!attr_ok) { cudaGetLastError(); return W4A4_ERR_CUDA; }
   d.ok = true;
@@ -464,6 +468,10 @@ int launch_gemm_cfg(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, con
   p.ldq = 0;
   p.next_K = 0;
   p.q_col0 = 0;
+  p.n_rope = 0;
+  p.d_head = 0;
+  p.rope = nullptr;
+  p.ld_rope = 0;
   const int64_t tiles = ceil_div(M, C::BM) * ceil_div(N, C::BN);
   const int64_t grid = tiles < dev->num_sms ? tiles : dev->num_sms;
   cudaLaunchConfig_t cfg = {};
@@ -491,14 +499,21 @@ struct QuantNext {
   int64_t ldq = 0, K = 0, col = 0;
 };
 
+// Rotary embedding of the leading plain outputs (n_rope == 0: off).
+struct RopeArgs {
+  int64_t n_rope = 0, d_head = 0, ld = 0;
+  const float* table = nullptr;
+};
+
 // The CTA-pair kernels: 256 x BN tiles on two SMs (cluster of 2).
 template <class C>
 int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
                      int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
                      const void* bias, int epi, void* Y, int64_t ldy, const float* next_inv_s, unsigned* next_amax,
                      cudaStream_t stream, DeviceInfo* dev, int64_t n_plain = -1, void* H = nullptr,
-                     int64_t ldh = 0, QuantNext qn = QuantNext()) {
+                     int64_t ldh = 0, QuantNext qn = QuantNext(), RopeArgs ra = RopeArgs()) {
   if (n_plain < 0) n_plain = N;
+  if (ra.n_rope > 0 && !C::ROPE) return W4A4_ERR_ARG;
   // SwiGLU outputs fill 32-column boxes from two 32-column accumulator blocks
   if (n_plain < N && (C::BN % 64 != 0 || n_plain % C::BN != 0)) return W4A4_ERR_SHAPE;
   CUtensorMap ta, tb, tsa, tsb, tu, tl, ty, th;
@@ -569,6 +584,10 @@ int launch_gemm_pair(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   p.ldq = qn.ldq;
   p.next_K = static_cast<int>(qn.K);
   p.q_col0 = static_cast<int>(qn.col);
+  p.n_rope = static_cast<int>(ra.n_rope);
+  p.d_head = static_cast<int>(ra.d_head);
+  p.rope = ra.table;
+  p.ld_rope = ra.ld;
   const int64_t tiles = ceil_div(M, 2 * C::BM) * ceil_div(N, C::BN);
   const int64_t max_pairs = dev->num_sms / 2;
   const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -763,6 +782,39 @@ int w4a4_gemm_swiglu(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
   return launch_gemm_pair<PairMain>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, W4A4_EPI_NONE, Y, ldy,
                                     next_inv_s, reinterpret_cast<unsigned*>(next_amax),
                                     static_cast<cudaStream_t>(stream), dev, n_plain, H, ldh);
+}
+
+int w4a4_gemm_rope(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M, int64_t N,
+                   int64_t K, const uint8_t* Wq, const uint8_t* Wsf, const float* t_w, const void* L2t, int r,
+                   const void* bias, int64_t n_rope, int64_t d_head, const float* rope, int64_t ld_rope,
+                   int64_t n_plain, void* Y, int64_t ldy, void* H, int64_t ldh, const float* next_inv_s,
+                   float* next_amax, void* stream) {
+  if (n_plain < 0 || n_plain > N || (n_plain < N && (n_plain % 256 != 0 || (N - n_plain) % 32 != 0)))
+    return W4A4_ERR_SHAPE;
+  if (d_head < 32 || d_head % 32 != 0 || n_rope <= 0 || n_rope % d_head != 0 || n_rope > n_plain ||
+      ld_rope < d_head || ld_rope % 4 != 0 || ld_rope > (int64_t(1) << 30))
+    return W4A4_ERR_SHAPE;
+  const bool swiglu = n_plain < N;
+  if (swiglu && (ldh < (N - n_plain) / 2 || ldh % 8 != 0)) return W4A4_ERR_SHAPE;
+  if (ldy < n_plain || ldy % 8 != 0) return W4A4_ERR_SHAPE;
+  int st = check_gemm_args(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, W4A4_EPI_NONE, Y, N);
+  if (st != W4A4_OK || M == 0) return st;
+  if (!rope || (swiglu && !H)) return W4A4_ERR_NULL;
+  if (!aligned16(rope) || (swiglu && !aligned16(H)) || (next_inv_s && !aligned16(next_inv_s)) ||
+      reinterpret_cast<uintptr_t>(next_amax) % 4 != 0)
+    return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  RopeArgs ra;
+  ra.n_rope = n_rope;
+  ra.d_head = d_head;
+  ra.ld = ld_rope;
+  ra.table = rope;
+  return launch_gemm_pair<PairRope>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, W4A4_EPI_NONE, Y, ldy,
+                                    next_inv_s, reinterpret_cast<unsigned*>(next_amax),
+                                    static_cast<cudaStream_t>(stream), dev, n_plain, swiglu ? H : nullptr, ldh,
+                                    QuantNext(), ra);
 }
 
 int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U, int64_t M,

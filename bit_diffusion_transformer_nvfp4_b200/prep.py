@@ -71,3 +71,22 @@ def swiglu_row_order(n_plain: int, n_ff: int, device=None) -> torch.Tensor:
     up = n_plain + n_ff + 16 * blocks + i
     tail = torch.cat([gate, up], dim=1).reshape(-1)
     return torch.cat([torch.arange(n_plain, device=device), tail])
+
+
+def rope_table(pos: torch.Tensor, axes_dims, base: float = 10000.0) -> torch.Tensor:
+    """The table ``w4a4_gemm_rope`` reads, from integer token positions ``pos``
+    [M, n_axes]: per token, the (cos, sin) of each head feature pair,
+    interleaved, fp32 [M, sum(axes_dims)].  Axis a owns the next
+    axes_dims[a] / 2 pairs; pair j of the axis turns at base^(-2j /
+    axes_dims[a]) per unit of that axis's position (one axis: the rotary
+    embedding's usual schedule).  Built once per sequence layout, in fp64 and
+    rounded once to fp32, like the precomputed position embedding of a DiT."""
+    pos = pos.to(torch.float64)
+    if pos.dim() == 1:
+        pos = pos[:, None]
+    if pos.shape[1] != len(axes_dims) or any(d % 2 for d in axes_dims):
+        raise ValueError("one even feature count per position axis")
+    theta = torch.cat([pos[:, a:a + 1] * torch.pow(torch.tensor(float(base), dtype=torch.float64, device=pos.device),
+                                                   -torch.arange(0, d, 2, dtype=torch.float64, device=pos.device) / d)
+                       for a, d in enumerate(axes_dims)], dim=1)
+    return torch.stack([torch.cos(theta), torch.sin(theta)], dim=-1).reshape(pos.shape[0], -1).to(torch.float32)

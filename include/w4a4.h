@@ -263,6 +263,44 @@ int w4a4_gemm_swiglu(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, co
                      float* next_amax, void* stream);
 
 /*
+ * w4a4_gemm_rope -- w4a4_gemm_swiglu whose epilogue also applies the rotary
+ * position embedding to the leading query/key features, the third epilogue
+ * the NVIDIA blog page on FLUX on Blackwell names for its fused NVFP4 GEMM
+ * ("NVIDIA Technical Blog Details FLUX 3 Image Klein Blackwell Inference
+ * Optimization Methods", the NVFP4 / fused-GEMM paragraph: SwiGLU, QKV
+ * projection and RoPE epilogues).  The page gives no formula; this is the
+ * rotation of adjacent feature pairs by per-token, per-pair angles given as a
+ * table (any 1-D or multi-axis angle schedule reduces to one).  Rows n <
+ * n_rope form n_rope / d_head heads of d_head features; in every head,
+ * features 2i and 2i+1 (i = 0 .. d_head/2 - 1) are the pair i.  With y as in
+ * w4a4_gemm_swiglu (fp32, t_x t_w acc + bias) and, for token m and pair i,
+ * c = rope[m * ld_rope + 2i], s = rope[m * ld_rope + 2i + 1]
+ * (cos and sin of its angle):
+ *   Y[m, head + 2i]     = bf16(y[m, head + 2i] c - y[m, head + 2i + 1] s)
+ *   Y[m, head + 2i + 1] = bf16(y[m, head + 2i] s + y[m, head + 2i + 1] c)
+ * one rounding of the rotated fp32 value (the values are not rounded to bf16
+ * before the rotation).  Rows n_rope <= n < n_plain are plain outputs, rows
+ * n >= n_plain SwiGLU pairs, exactly as in w4a4_gemm_swiglu.  Same arguments
+ * as w4a4_gemm_swiglu plus
+ *   n_rope      rotated features, 0 < n_rope <= n_plain, a multiple of d_head
+ *   d_head      features per head, a multiple of 32
+ *   rope        in fp32 [M, ld_rope]: per token the d_head/2 (cos, sin) pairs
+ *               of its head features, the same for every head; 16-byte aligned
+ *   ld_rope     row stride of rope in floats, >= d_head, a multiple of 4
+ * and n_plain may equal N (no SwiGLU features; H NULL, next_amax over Y).
+ * With n_plain < N it must be a multiple of 256, as in w4a4_gemm_swiglu.
+ * W4A4_ERR_SHAPE for sizes outside these ranges, W4A4_ERR_NULL for a NULL
+ * rope, W4A4_ERR_ALIGN for a misaligned one.  Launches one CTA-pair GEMM
+ * kernel.
+ */
+int w4a4_gemm_rope(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, const void* U,
+                   int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,
+                   const float* t_w, const void* L2t, int r, const void* bias,
+                   int64_t n_rope, int64_t d_head, const float* rope, int64_t ld_rope,
+                   int64_t n_plain, void* Y, int64_t ldy, void* H, int64_t ldh,
+                   const float* next_inv_s, float* next_amax, void* stream);
+
+/*
  * w4a4_gemm_quantize_next -- w4a4_gemm (epilogue NONE or GELU_TANH) or
  * w4a4_gemm_swiglu (n_plain < N) whose epilogue also quantises its final
  * outputs for the next layer, so that layer's activation quantiser need not

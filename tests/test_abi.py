@@ -206,6 +206,31 @@ def test_swiglu_argument_checks(so):
              None, None, None) == 0
 
 
+def test_rope_argument_checks(so):
+    """w4a4_gemm_rope rejects bad head sizes, table strides and pointers on the host."""
+    P = 1 << 20
+
+    def call(n_rope=256, d_head=128, rope=P, ld_rope=128, n_plain=512, N=768, H=P, ldh=128, M=128):
+        #                Xq Xsf t_x U  M  N  K    Wq Wsf t_w L2t  r  bias
+        return so.w4a4_gemm_rope(P, P, P, None, M, N, 512, P, P, P, None, 0, None,
+                                 n_rope, d_head, rope, ld_rope, n_plain, P, n_plain, H, ldh, None, None, None)
+    if not __import__("torch").cuda.is_available():
+        assert call() == -4                                  # valid: reaches the device check
+        assert call(N=512, H=None, ldh=0) == -4              # no SwiGLU features
+        assert call(d_head=32, ld_rope=36) == -4             # padded table rows
+    assert call(d_head=48, n_rope=240, ld_rope=48) == -2     # head size not a multiple of 32
+    assert call(n_rope=192) == -2                            # not a whole number of heads
+    assert call(n_rope=0) == -2                              # nothing to turn: use w4a4_gemm_swiglu
+    assert call(n_rope=768, n_plain=512) == -2               # beyond the plain features
+    assert call(ld_rope=96) == -2                            # table row shorter than a head
+    assert call(ld_rope=130) == -2                           # table rows not 16-byte aligned
+    assert call(n_plain=384) == -2                           # SwiGLU split not a multiple of 256
+    assert call(rope=None) == -1
+    assert call(rope=P + 4) == -3
+    assert call(H=None) == -1                                # SwiGLU features need H
+    assert call(M=0, rope=None) == 0                         # empty problem
+
+
 def test_quantize_next_argument_checks(so):
     """w4a4_gemm_quantize_next rejects bad column ranges, strides and pointers on the host."""
     P = 1 << 20

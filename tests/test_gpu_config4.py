@@ -172,3 +172,44 @@ def test_config4_swiglu_full_size(w4, layers):
         h = from_dev_bf16(H[r0:r0 + 2048])
         want = max(want, np.float32(np.max(np.abs((h * s_next[None, :]).astype(np.float32)))))
     assert got == float(want)
+
+
+def test_config4_rope_swiglu_full_size(w4, layers):
+    """The fused projection with all three epilogues at 16896 tokens: the
+    rotary embedding on the 2 x 6144 query and key features (heads of 128,
+    angles of the text + 128 x 128 image-token sequence), V plain, SwiGLU on
+    the rest.  Sampled tokens x sampled whole heads against the oracle; V and
+    H bit for bit equal to the SwiGLU kernel's (the same epilogue there)."""
+    import torch
+    from bit_diffusion_transformer_nvfp4_b200 import prep as gprep
+    from oracle import rope as orope
+    from synth import token_positions
+    c, p, _ = layers[0]
+    n_plain = n_ff = 18432
+    n_rope, d_head, axes = 12288, 128, (16, 56, 56)
+    perm = gprep.swiglu_row_order(n_plain, n_ff).numpy()
+    pw = w4.pack_weight(to_dev_f32(p["R"][perm]))
+    w = w4.PackedWeight(pw.Wq, pw.Wsf, pw.t_w, c.N, c.K, to_dev_f32(p["inv_s"]), to_dev_bf16(p["L1t"]),
+                        to_dev_bf16(p["L2t"][perm]), None)
+    qa = w4.quantize_act(to_dev_bf16(c.x), w.inv_s, w.L1t, w.t_w)
+    tab = orope.table(orope.angles(token_positions(512, 128, 128), axes, 10000.0))
+    assert tab.shape == (c.M, d_head)
+    Y0, H0 = w4.gemm_swiglu(qa, w, n_plain)
+    Y, H = w4.gemm_rope(qa, w, torch.from_numpy(tab).cuda(), n_rope, d_head, n_plain=n_plain)
+    torch.cuda.synchronize()
+    assert w4.w4a4_device_status() == 0
+    assert torch.equal(H.view(torch.int16), H0.view(torch.int16))
+    assert torch.equal(Y[:, n_rope:].view(torch.int16), Y0[:, n_rope:].view(torch.int16))
+
+    g = rng(46)
+    rows = np.sort(g.choice(c.M, 64, replace=False))
+    rows[0], rows[-1] = 0, c.M - 1                       # a text token and the last image token
+    heads = np.sort(g.choice(n_rope // d_head, 6, replace=False))
+    heads[-1] = n_rope // d_head - 1
+    cols = (heads[:, None] * d_head + np.arange(d_head)[None, :]).reshape(-1)
+    oq, osf, ot, _ = nvfp4.quantize(p["R"][cols], amax=np.max(np.abs(p["R"])))
+    y_ref, _ = olinear.w4a4_linear(c.x, p["inv_s"], nvfp4.pack(oq), osf, ot, p["L1t"], p["L2t"][cols], None,
+                                   rows=rows)
+    want = orope.rotate(y_ref, tab[rows], len(cols), d_head)
+    got = from_dev_bf16(Y[torch.from_numpy(rows).cuda()])[:, cols]
+    check_y(got, want)
