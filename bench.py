@@ -695,6 +695,29 @@ def run_table(args):
               "gemm_with_next_codes_us": round(t_store, 2), "gemm_next_codes_only_us": round(t_codes, 2),
               "gemm_next_codes_only_tflops": tf(gfl, t_codes)})
 
+    def rope_row(cfg, case, pk, qa, g, n_plain, d_head=128, axes=(16, 56, 56), n_text=512, side=128):
+        """The fused projection with the rotary embedding on its query and key
+        features (w4a4_gemm_rope; heads of 128, the angles of a text + image
+        token sequence) beside the same GEMM with the SwiGLU epilogue alone."""
+        from synth import token_positions
+        M, N = qa.M, pk.N
+        n_rope = 2 * (n_plain // 3)                  # Q and K of the plain Q | K | V features
+        tab = prep.rope_table(torch.from_numpy(token_positions(n_text, side, side)).to(dev), axes)
+        assert tab.shape[0] == M
+        Y = torch.empty(M, n_plain, dtype=torch.bfloat16, device=dev)
+        H = torch.empty(M, (N - n_plain) // 2, dtype=torch.bfloat16, device=dev)
+
+        def gr():
+            w4.gemm_rope(qa, pk, tab, n_rope, d_head, n_plain=n_plain, Y=Y, H=H)
+        t_plain, t_rope = med_us([g, gr])
+        check()
+        gfl = gemm_flops(M, case.K, N, pk.r)
+        emit({"table": "rope_epilogue", "config": cfg, "layer": case.name, "M": M, "K": case.K, "N": N,
+              "rotated_outputs": n_rope, "d_head": d_head, "gemm_swiglu_us": round(t_plain, 2),
+              "gemm_rope_swiglu_us": round(t_rope, 2), "gemm_rope_swiglu_tflops": tf(gfl, t_rope),
+              "gemm_rope_swiglu_frac_fp4": round(tf(gfl, t_rope) / fp4_peak, 3),
+              "rope_cost_pct": round(100.0 * (t_rope / t_plain - 1.0), 2)})
+
     emit({"table": "peaks", "fp4_peak_tflops": round(fp4_peak, 1), "hbm_gbs": peaks["hbm_gbs"],
           "basis": f"{peak_kind}: bf16 burst x {FP4_OVER_BF16:g}; copy bandwidth", "reps": reps,
           "l2": "256 MB buffer zeroed before each repetition"})
@@ -743,6 +766,7 @@ def run_table(args):
             if cfg == 1:
                 graph_row(case, pk, X, qa, ws, Y, qi, g)
             if n_plain is not None:
+                rope_row(cfg, case, pk, qa, g, n_plain)
                 quant_next_row(cfg, case, pk, qa, g, n_plain=n_plain, next_K=24576, next_col=6144)
             del pk, X, qa, ws, Y
             torch.cuda.empty_cache()
@@ -857,6 +881,9 @@ CASES = {
     "gemm_block2048_up": ("w4a4_gemm_swiglu, the 2048px fused QKV+SwiGLU-up projection", 16896, 6144, 55296, 18432),
     "gemm_block2048_up_small": ("w4a4_gemm_swiglu, the 2048px fused projection at 4096 tokens", 4096, 6144, 55296, 18432),
     "gemm_block2048_out": ("w4a4_gemm, the 2048px output projection", 16896, 24576, 6144, None),
+    "gemm_rope_block2048_small": ("w4a4_gemm_rope, the 2048px fused projection at 4096 tokens, the rotary embedding "
+                                  "on its 12288 query and key outputs (heads of 128) and SwiGLU on the rest",
+                                  4096, 6144, 55296, 18432),
     "gemm_quant_next_block2048_small": ("w4a4_gemm_quantize_next, the 2048px fused projection at 4096 tokens, its "
                                         "SwiGLU outputs quantised into columns 6144.. of a 24576-wide activation",
                                         4096, 6144, 55296, 18432),
@@ -927,6 +954,15 @@ def run_case(args):
                     w4.w4a4_gemm_quantize_next(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, pw.Wq, pw.Wsf, pw.t_w, L2t, r,
                                                None, 0, n_plain, Y, n_plain, H, H.shape[1], None, t_next, nq,
                                                nq.stride(0), nsf, 24576, 6144, None, st)
+            elif args.case.startswith("gemm_rope"):
+                Y = torch.empty(M, n_plain, dtype=torch.bfloat16, device=dev)
+                H = torch.empty(M, (N - n_plain) // 2, dtype=torch.bfloat16, device=dev)
+                from bit_diffusion_transformer_nvfp4_b200 import prep
+                tab = prep.rope_table(torch.arange(M, device=dev), (128,))   # one position axis
+
+                def call():
+                    w4.w4a4_gemm_rope(qa.Xq, qa.Xsf, qa.t_x, qa.U, M, N, K, pw.Wq, pw.Wsf, pw.t_w, L2t, r, None,
+                                      12288, 128, tab, 128, n_plain, Y, n_plain, H, H.shape[1], None, None, st)
             elif n_plain is None:
                 Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
 

@@ -237,10 +237,45 @@ __device__ __forceinline__ float tensor_scale_from(float amax) {
   return t;
 }
 
+// Columns 16hh .. 16hh+15 of a row's low-rank sum, scaled by ra = 1/(t_x t_w),
+// as the bf16 hi|lo pair (row of 2r bf16: hi in columns [0, r), lo in [r, 2r)).
+__device__ __forceinline__ void store_lowrank16(const QuantParams& p, float ra, __nv_bfloat16* urow, int hh,
+                                                const float (&acc)[16]) {
+  uint32_t hi[8], lo[8];
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
+    const uint32_t h = pack_bf16x2(a0, a1);
+    hi[j / 2] = h;
+    lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
+  }
+  uint4* dh = reinterpret_cast<uint4*>(urow + 16 * hh);
+  uint4* dl = reinterpret_cast<uint4*>(urow + p.r + 16 * hh);
+  dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  dh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+  dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+}
+
+// A row block covered by one piece: its U is final in TMEM; the row's sum is
+// 0 + u (the same arithmetic as the sum of one partial), no round trip.
+__device__ __forceinline__ void store_lowrank_row(const QuantParams& p, float ra, int64_t row,
+                                                  const uint32_t (&u)[32]) {
+  __nv_bfloat16* urow = p.u_out + row * 2 * p.r;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {  // r = 16 or 32: one or two groups of 16 columns
+    if (hh < p.r / 16) {
+      float acc[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) acc[j] = __fadd_rn(0.0f, __uint_as_float(u[16 * hh + j]));
+      store_lowrank16(p, ra, urow, hh, acc);
+    }
+  }
+}
+
 // The last K slice of a row block sums the fp32 partials in slice order,
-// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row (row of 2r
-// bf16: hi in columns [0, r), lo in [r, 2r); columns in groups of 16, two
-// slices' loads in flight).
+// scales by 1/(t_x t_w) and writes the bf16 hi|lo pair of its row (columns
+// in groups of 16, two slices' loads in flight).
 __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, int64_t rows_pad, int64_t prow,
                                                  int64_t row, int n_parts) {
   __threadfence();
@@ -275,22 +310,7 @@ __device__ __forceinline__ void finalize_lowrank(const QuantParams& p, float t, 
         }
       }
     }
-    if (row < p.M) {
-      uint32_t hi[8], lo[8];
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        const float a0 = __fmul_rn(acc[j], ra), a1 = __fmul_rn(acc[j + 1], ra);
-        const uint32_t h = pack_bf16x2(a0, a1);
-        hi[j / 2] = h;
-        lo[j / 2] = pack_bf16x2(__fsub_rn(a0, bf16_lo(h)), __fsub_rn(a1, bf16_hi(h)));
-      }
-      uint4* dh = reinterpret_cast<uint4*>(urow + 16 * hh);
-      uint4* dl = reinterpret_cast<uint4*>(urow + p.r + 16 * hh);
-      dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      dh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-      dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-    }
+    if (row < p.M) store_lowrank16(p, ra, urow, hh, acc);
   }
 }
 
@@ -476,6 +496,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
       const int quarter = warp & 3;  // the TMEM lane quarter this warp may read
       const int ut = (warp - kQUWarp0) * 32 + lane;
       const int64_t rows_pad = static_cast<int64_t>(p.row_blocks) * kQRows;
+      const float ra_u = __frcp_rn(__fmul_rn(t, __ldg(p.t_w)));
       int j = 0;
       for (int64_t g = g_begin; g < g_end; g += piece_at(g).n, ++j) {
         const int a = j % kQAcc;
@@ -493,6 +514,10 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_kernel(const __grid_consta
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&acc_empty[a]));
         const int64_t prow = static_cast<int64_t>(rb) * kQRows + quarter * 32 + lane;
+        if (n_parts == 1) {
+          if (prow < p.M) store_lowrank_row(p, ra_u, prow, u);
+          continue;
+        }
         float4* dst = reinterpret_cast<float4*>(p.u_part + (static_cast<int64_t>(split) * rows_pad + prow) * 32);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
