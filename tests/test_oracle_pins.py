@@ -517,3 +517,76 @@ def test_rope_scores_depend_only_on_relative_position():
     s0 = score([0, 3, 9], [0, 1, 4])
     assert abs(score([5, 10, 12], [5, 8, 7]) - s0) < 1e-5
     assert abs(score([0, 4, 9], [0, 1, 4]) - s0) > 1e-3           # a different offset does change it
+
+
+# ---------------------------------------------------------------- FP8 attention
+
+@pytest.mark.parametrize("v,byte", [
+    (1.0, 0x38), (-1.0, 0xB8), (448.0, 0x7E), (500.0, 0x7E), (-1e6, 0xFE), (0.0, 0x00), (-0.0, 0x80),
+    (2.0 ** -9, 0x01), (-2.0 ** -9, 0x81), (2.0 ** -11, 0x00), (1.0625, 0x38), (1.1875, 0x3A), (0.875, 0x36),
+    (240.0, 0x77), (3.0 * 2.0 ** -9, 0x03), (2.5 * 2.0 ** -9, 0x02),
+])
+def test_fp8_signed_encoding_by_hand(v, byte):
+    from oracle import attention
+    assert int(attention.e4m3_encode(np.array([v], np.float32))[0]) == byte
+
+
+def test_fp8_encoding_against_library():
+    torch = pytest.importorskip("torch")
+    from oracle import attention
+    g = rng(51)
+    x = np.concatenate([g.standard_normal(4000) * 30.0, g.standard_normal(1000) * 0.01,
+                        np.array([447.9, -447.9, 2.0 ** -10, -2.0 ** -10])]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(attention.e4m3_encode(x), want)
+
+
+def test_fp8_tensor_quantiser():
+    from oracle import attention
+    g = rng(52)
+    x = bf16_round(g.standard_normal((64, 48)).astype(np.float32) * 5.0)
+    codes, s = attention.fp8_quantize(x)
+    assert s == np.float32(np.float32(np.max(np.abs(x))) / np.float32(448.0))
+    i = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert codes[i] & 0x7F == 0x7E                               # the largest element takes the largest code
+    back = attention.fp8_dequantize(codes, s)
+    assert np.all(np.abs(back - x) <= np.abs(x) * 2.0 ** -4 + float(s) * 2.0 ** -10)   # half an E4M3 step
+    z, s0 = attention.fp8_quantize(np.zeros((3, 4), np.float32))
+    assert s0 == 1.0 and not np.any(z)
+
+
+def test_attention_two_keys_by_hand():
+    from oracle import attention
+    # scores (ln 3, 0): weights 3/4 and 1/4
+    q = np.array([[1.0, 0.0]])
+    k = np.array([[np.log(3.0), 0.0], [0.0, 0.0]])
+    v = np.array([[4.0, -8.0], [8.0, 4.0]])
+    o = attention.attention(q, k, v, heads=1, scale=1.0)
+    np.testing.assert_allclose(o, [[0.75 * 4 + 0.25 * 8, 0.75 * -8 + 0.25 * 4]], rtol=1e-14)
+
+
+def test_attention_closed_forms():
+    from oracle import attention
+    g = rng(53)
+    S, H, d = 24, 2, 8
+    q = g.standard_normal((S, H * d))
+    k = g.standard_normal((S, H * d))
+    v = g.standard_normal((S, H * d))
+    o = attention.attention(q, k, v, H)
+    # identical keys: every query averages the values
+    o_u = attention.attention(q, np.ones_like(k), v, H)
+    np.testing.assert_allclose(o_u, np.broadcast_to(v.mean(axis=0), o_u.shape), rtol=1e-12)
+    # keys and values permuted together: unchanged; queries permuted: rows permuted
+    perm = g.permutation(S)
+    np.testing.assert_allclose(attention.attention(q, k[perm], v[perm], H), o, rtol=1e-12)
+    np.testing.assert_allclose(attention.attention(q[perm], k, v, H), o[perm], rtol=1e-12)
+    # heads are independent
+    np.testing.assert_allclose(o[:, d:], attention.attention(q[:, d:], k[:, d:], v[:, d:], 1,
+                                                             scale=1.0 / np.sqrt(d)), rtol=1e-12)
+    # one dominant key selects its value; huge scores do not overflow
+    k2 = k.copy()
+    k2[5] = 1e4 * q[0]
+    o2 = attention.attention(q[:1], k2, v, H)
+    np.testing.assert_allclose(o2[0], v[5], atol=1e-12)
+    # the scale of the scores is 1/sqrt(d) by default
+    np.testing.assert_allclose(attention.attention(q, k, v, H, scale=1.0 / np.sqrt(d)), o, rtol=1e-15)
