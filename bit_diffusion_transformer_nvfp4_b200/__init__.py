@@ -13,6 +13,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import math
+
 import torch
 
 __all__ = [
@@ -23,6 +25,7 @@ __all__ = [
     "new_workspace", "nvfp4_sf_to_rowmajor", "sf_rowmajor", "w4a4_set_wait_bound",
     "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
     "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next", "w4a4_gemm_rope", "gemm_rope",
+    "fp8_quant_workspace_bytes", "fp8_quantize", "attention_fp8", "Fp8Tensor", "quantize_fp8", "attention",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -51,6 +54,10 @@ _SIG = {
                                     _P, _I64, _P, _P, _P]),
     "w4a4_gemm_rope": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _I64, _I64, _P,
                                   _I64, _I64, _P, _I64, _P, _I64, _P, _P, _P]),
+    "fp8_quant_workspace_bytes": (_c.c_size_t, [_I64, _I64]),
+    "fp8_quantize": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_int, _P, _I64, _P, _P, _c.c_size_t, _P]),
+    "attention_fp8": (_c.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _c.c_float, _P, _I64,
+                                 _P]),
     "w4a4_gemm_quantize_next": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P,
                                            _c.c_int, _I64, _P, _I64, _P, _I64, _P, _P, _P, _I64, _P, _I64, _I64,
                                            _P, _P]),
@@ -172,6 +179,22 @@ def w4a4_gemm_rope(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_rope,
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), n_rope, d_head, _ptr(rope), ld_rope, n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s),
         _ptr(next_amax), _stream(stream)))
+
+
+def fp8_quant_workspace_bytes(rows, cols) -> int:
+    return lib().fp8_quant_workspace_bytes(rows, cols)
+
+
+def fp8_quantize(X, rows, cols, ldx, transpose, out, ldo, scale, workspace, stream=None):
+    _check("fp8_quantize", lib().fp8_quantize(
+        _ptr(X), rows, cols, ldx, int(transpose), _ptr(out), ldo, _ptr(scale), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def attention_fp8(Q8, K8, Vt8, batch, S, heads, ldq, ldk, ldvt, s_q, s_k, s_v, softmax_scale, O, ldo, stream=None):
+    _check("attention_fp8", lib().attention_fp8(
+        _ptr(Q8), _ptr(K8), _ptr(Vt8), batch, S, heads, ldq, ldk, ldvt, _ptr(s_q), _ptr(s_k), _ptr(s_v),
+        float(softmax_scale), _ptr(O), ldo, _stream(stream)))
 
 
 def w4a4_gemm_quantize_next(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, n_plain, Y, ldy, H,
@@ -349,6 +372,42 @@ def gemm_rope(qa: QuantizedActivation, w: PackedWeight, rope, n_rope: int, d_hea
                    d_head, rope, rope.stride(0), n_plain, Y, Y.stride(0), H, 0 if H is None else H.stride(0),
                    next_inv_s, next_amax, stream)
     return Y, H
+
+
+class Fp8Tensor:
+    """E4M3 codes of a bf16 tensor and its fp32 scale (row-major, or
+    transposed when ``transposed``)."""
+
+    def __init__(self, codes, scale, rows, cols, transposed):
+        self.codes, self.scale, self.rows, self.cols, self.transposed = codes, scale, rows, cols, transposed
+
+
+def quantize_fp8(X, transpose: bool = False, out=None, workspace=None, stream=None) -> Fp8Tensor:
+    """Per-tensor E4M3 quantisation of a bf16 [rows, cols] view (row stride
+    X.stride(0)); transposed codes [cols, rows] with ``transpose``."""
+    rows, cols = X.shape
+    dev = X.device
+    if out is None:
+        out = torch.empty((cols, rows) if transpose else (rows, cols), dtype=torch.uint8, device=dev)
+    scale = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(fp8_quant_workspace_bytes(rows, cols), 16), dtype=torch.uint8, device=dev)
+    fp8_quantize(X, rows, cols, X.stride(0), transpose, out, out.stride(0), scale, workspace, stream)
+    return Fp8Tensor(out, scale, rows, cols, transpose)
+
+
+def attention(q: Fp8Tensor, k: Fp8Tensor, vt: Fp8Tensor, heads: int, batch: int = 1, O=None, softmax_scale=None,
+              stream=None):
+    """FP8 attention over ``batch`` sequences of q.rows / batch tokens, heads
+    of 128 features; q, k row-major codes [tokens, heads*128], vt the values'
+    transposed codes [heads*128, tokens].  Returns bf16 O [tokens, heads*128]."""
+    S = q.rows // batch
+    if O is None:
+        O = torch.empty(q.rows, heads * 128, dtype=torch.bfloat16, device=q.codes.device)
+    c = 1.0 / math.sqrt(128.0) if softmax_scale is None else softmax_scale
+    attention_fp8(q.codes, k.codes, vt.codes, batch, S, heads, q.codes.stride(0), k.codes.stride(0),
+                  vt.codes.stride(0), q.scale, k.scale, vt.scale, c, O, O.stride(0), stream)
+    return O
 
 
 def gemm_quantize_next(qa: QuantizedActivation, w: PackedWeight, next_t, next_inv_s=None, epilogue: int = EPI_NONE,

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libw4a4.so")
 SOURCES = ["w4a4_api.cu"]
-DEPS = ["w4a4_api.cu", "gemm.cuh", "gemm2.cuh", "quant.cuh", "sm100.cuh"]
+DEPS = ["w4a4_api.cu", "attention.cuh", "gemm.cuh", "gemm2.cuh", "quant.cuh", "sm100.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -44,6 +44,8 @@ def up_to_date() -> bool:
         return False
     t = os.path.getmtime(LIB)
     deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", "w4a4.h")]
+    # every source in csrc/ counts, listed or not
+    deps += [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 

@@ -158,16 +158,6 @@ struct GemmCfg {
 // the epilogue the bottleneck).  The hardware base-2 exponential and
 // reciprocal keep the result within a few fp32 ulps, far inside the bf16
 // rounding of the output.
-__device__ __forceinline__ float ex2_approx(float x) {
-  float r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
 __device__ __forceinline__ float gelu_tanh_f32(float y) {
   const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
   const float t = ex2_approx(-2.8853900817779268f * fabsf(u));  // exp(-2|u|) = 2^(-2 log2(e) |u|)

@@ -17,6 +17,7 @@
 #include "gemm2.cuh"
 
 #include "quant.cuh"
+#include "attention.cuh"
 
 namespace w4a4 {
 
@@ -88,6 +89,8 @@ int device_setup(DeviceInfo** out) {
                                   QuantTile<float>::kSmem) == cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(quant_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   FusedQuantSmem::kBytes) == cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::kBytes) ==
+             cudaSuccess;
   using G256 = GemmCfg<256, 4>;
   using G192 = GemmCfg<192, 4>;
 
@@ -853,6 +856,118 @@ int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* 
   return launch_gemm_pair<PairQNext>(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, epilogue, Y, ldy,
                                      next_inv_s, reinterpret_cast<unsigned*>(next_amax),
                                      static_cast<cudaStream_t>(stream), dev, n_plain, H, ldh, qn);
+}
+
+size_t fp8_quant_workspace_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols <= 0 || cols % 8 != 0) return 0;
+  return sizeof(float) * kAmaxMaxBlocks;  // the tensor-amax partial maxima
+}
+
+int fp8_quantize(const void* X, int64_t rows, int64_t cols, int64_t ldx, int transpose, uint8_t* out, int64_t ldo,
+                 float* scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (transpose != 0 && transpose != 1) return W4A4_ERR_ARG;
+  if (rows < 0 || cols <= 0 || cols % 8 != 0 || ldx < cols || ldx % 8 != 0 || rows > (int64_t(1) << 30) ||
+      cols > (int64_t(1) << 30))
+    return W4A4_ERR_SHAPE;
+  if (transpose ? (rows % 16 != 0 || ldo < rows || ldo % 16 != 0) : (ldo < cols || ldo % 8 != 0))
+    return W4A4_ERR_SHAPE;
+  if (rows == 0) return W4A4_OK;  // empty tensor: nothing enqueued
+  if (!X || !out || !scale) return W4A4_ERR_NULL;
+  if (!aligned16(X) || !aligned16(out) || reinterpret_cast<uintptr_t>(scale) % 4 != 0 ||
+      (workspace && !aligned16(workspace)))
+    return W4A4_ERR_ALIGN;
+  if (!workspace || workspace_bytes < fp8_quant_workspace_bytes(rows, cols)) return W4A4_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  float* partials = static_cast<float*>(workspace);
+  // pass 1: the tensor amax (column-segment CTAs times row bands, as for the activations)
+  const int64_t gx = ceil_div(cols / 8, kAmaxThreads);
+  int64_t gy = ceil_div(4 * static_cast<int64_t>(dev->num_sms), gx);
+  if (gy > kAmaxMaxBlocks / gx) gy = kAmaxMaxBlocks / gx;
+  if (gy > rows) gy = rows;
+  if (gy < 1) gy = 1;
+  const int64_t rows_per = ceil_div(rows, gy);
+  gy = ceil_div(rows, rows_per);
+  amax_kernel<__nv_bfloat16><<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kAmaxThreads, 0, strm>>>(
+      static_cast<const __nv_bfloat16*>(X), rows, cols, ldx, nullptr, partials, static_cast<int>(rows_per));
+  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  // pass 2: codes, 128 x 64 tiles
+  Fp8QuantParams p;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.rows = rows;
+  p.cols = cols;
+  p.ldx = ldx;
+  p.out = out;
+  p.ldo = ldo;
+  p.partials = partials;
+  p.n_partials = static_cast<int>(gx * gy);
+  p.scale_out = scale;
+  p.transpose = transpose;
+  const int64_t ty = ceil_div(rows, 128);
+  if (ty > 65535) return W4A4_ERR_SHAPE;
+  fp8_quant_kernel<<<dim3(static_cast<unsigned>(ceil_div(cols, 64)), static_cast<unsigned>(ty)), 256, 0, strm>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;
+  return W4A4_OK;
+}
+
+int attention_fp8(const uint8_t* Q8, const uint8_t* K8, const uint8_t* Vt8, int64_t batch, int64_t S, int64_t heads,
+                  int64_t ldq, int64_t ldk, int64_t ldvt, const float* s_q, const float* s_k, const float* s_v,
+                  float softmax_scale, void* O, int64_t ldo, void* stream) {
+  if (batch < 0 || S < 0 || heads <= 0 || S % kAttnTile != 0 || heads > 65535 || batch > 65535 ||
+      S > (int64_t(1) << 24))
+    return W4A4_ERR_SHAPE;
+  const int64_t width = heads * kAttnD;
+  if (ldq < width || ldq % 16 != 0 || ldk < width || ldk % 16 != 0 || ldvt < batch * S || ldvt % 16 != 0 ||
+      ldo < width || ldo % 8 != 0)
+    return W4A4_ERR_SHAPE;
+  if (!(softmax_scale > 0.0f) || !(softmax_scale < 3.0e38f)) return W4A4_ERR_ARG;
+  if (batch == 0 || S == 0) return W4A4_OK;  // no tokens
+  if (!Q8 || !K8 || !Vt8 || !s_q || !s_k || !s_v || !O) return W4A4_ERR_NULL;
+  if (!aligned16(Q8) || !aligned16(K8) || !aligned16(Vt8) || !aligned16(O) ||
+      reinterpret_cast<uintptr_t>(s_q) % 4 != 0 || reinterpret_cast<uintptr_t>(s_k) % 4 != 0 ||
+      reinterpret_cast<uintptr_t>(s_v) % 4 != 0)
+    return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if (!encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q8, static_cast<uint64_t>(width),
+                 static_cast<uint64_t>(batch * S), static_cast<uint64_t>(ldq), 128u, 128u,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, K8, static_cast<uint64_t>(width),
+                 static_cast<uint64_t>(batch * S), static_cast<uint64_t>(ldk), 128u, 128u,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, Vt8, static_cast<uint64_t>(batch * S),
+                 static_cast<uint64_t>(width), static_cast<uint64_t>(ldvt), 128u, 128u,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return W4A4_ERR_CUDA;
+  AttnParams p;
+  p.S = static_cast<int>(S);
+  p.heads = static_cast<int>(heads);
+  p.s_q = s_q;
+  p.s_k = s_k;
+  p.s_v = s_v;
+  p.scale = softmax_scale;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.ldo = ldo;
+  p.status = dev->status_ptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(S / kAttnTile), static_cast<unsigned>(heads), static_cast<unsigned>(batch));
+  cfg.blockDim = dim3(kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = AttnSmem::kBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn_fp8_kernel, tq, tk, tv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  return W4A4_OK;
 }
 
 int w4a4_linear(const void* X, int64_t M, int64_t N, int64_t K, const uint8_t* Wq, const uint8_t* Wsf,

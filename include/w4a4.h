@@ -346,6 +346,59 @@ int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* 
                             float* next_amax, void* stream);
 
 /*
+ * FP8 attention.  The NVIDIA blog page on FLUX on Blackwell quantises the
+ * attention that consumes the fused projection's queries, keys and values to
+ * FP8 ("NVIDIA Technical Blog Details FLUX 3 Image Klein Blackwell Inference
+ * Optimization Methods", the paragraph on quantised and sparse attention:
+ * VC-Attention FP8) and states no arithmetic; the reading implemented here is
+ * per-tensor E4M3 quantisation of Q, K and V and the exact softmax attention
+ * of the dequantised tensors, evaluated on the FP8 tensor cores.  The page's
+ * "repair budget" is not defined there and is not implemented.
+ *
+ * fp8_quantize -- one bf16 tensor X [rows, cols] (row stride ldx elements) to
+ * E4M3 codes with one fp32 scale s = amax / 448 (1 when that is not a normal
+ * number), code = E4M3_rn_satfinite(fl(x * fl(1/s))), written row-major
+ * (out[r * ldo + c], transpose = 0) or transposed (out[c * ldo + r],
+ * transpose = 1: the value layout attention_fp8 reads).  Two kernels: the
+ * tensor amax into the workspace, then the codes.
+ *   cols % 8 == 0, ldx >= cols, ldx % 8 == 0; transpose: rows % 16 == 0,
+ *   ldo >= rows, ldo % 16 == 0; else ldo >= cols, ldo % 8 == 0
+ *   scale     out fp32 device scalar (4-byte aligned)
+ *   workspace >= fp8_quant_workspace_bytes(rows, cols) bytes of device memory
+ *             (no zeroing needed)
+ * W4A4_ERR_SHAPE / _NULL / _ALIGN / _WORKSPACE on bad arguments; rows == 0
+ * enqueues nothing.
+ */
+size_t fp8_quant_workspace_bytes(int64_t rows, int64_t cols);
+int fp8_quantize(const void* X, int64_t rows, int64_t cols, int64_t ldx, int transpose,
+                 uint8_t* out, int64_t ldo, float* scale, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/*
+ * attention_fp8 -- O = softmax(c Q K^T) V per head and sequence, on E4M3
+ * operands: batch sequences of S tokens (S % 128 == 0), heads of 128
+ * features.
+ *   Q8, K8  in  E4M3 [batch * S, ldq / ldk bytes], token-major, head h in
+ *               columns h*128 .. h*128+127 (ld >= heads*128, ld % 16 == 0)
+ *   Vt8     in  E4M3 [heads * 128, ldvt bytes]: V transposed, row h*128 + d,
+ *               column b*S + j (ldvt >= batch*S, ldvt % 16 == 0), as written
+ *               by fp8_quantize with transpose = 1
+ *   s_q, s_k, s_v  in fp32 device scalars: the tensors' dequantisation scales
+ *   softmax_scale  c (normally 1/sqrt(128)), finite and > 0
+ *   O       out bf16 [batch * S, ldo], head h in columns h*128 .. (ldo % 8 == 0)
+ * The kernel computes S = Q K^T on the tensor cores in fp32, an online
+ * softmax in fp32 with the probabilities rounded to E4M3 (within 2^-17 to
+ * 2^8.5 of the row's running maximum) for the second product O += P V, and
+ * writes bf16(O s_v / l), l the sum of the rounded probabilities.  One CTA
+ * per (128 queries, head, sequence), two per SM; programmatic stream
+ * serialisation as for the GEMMs.
+ */
+int attention_fp8(const uint8_t* Q8, const uint8_t* K8, const uint8_t* Vt8, int64_t batch, int64_t S,
+                  int64_t heads, int64_t ldq, int64_t ldk, int64_t ldvt, const float* s_q,
+                  const float* s_k, const float* s_v, float softmax_scale, void* O, int64_t ldo,
+                  void* stream);
+
+/*
  * w4a4_linear -- the whole hot path: nvfp4_quantize_act on X (row stride K)
  * into the workspace, then w4a4_gemm into Y (row stride N).
  *   workspace >= w4a4_workspace_bytes(M, N, K, r) bytes of device memory.

@@ -231,6 +231,35 @@ def test_rope_argument_checks(so):
     assert call(M=0, rope=None) == 0                         # empty problem
 
 
+def test_fp8_argument_checks(so):
+    """fp8_quantize and attention_fp8 reject bad sizes, strides and pointers on the host."""
+    P = 1 << 20
+    q = so.fp8_quantize
+    ws = so.fp8_quant_workspace_bytes(256, 256)
+    assert ws >= 4096 and so.fp8_quant_workspace_bytes(256, 250) == 0
+    #        X  rows cols ldx tr out ldo  scale ws  bytes stream
+    assert q(P, 256, 250, 256, 0, P, 256, P, P, ws, None) == -2          # cols % 8
+    assert q(P, 250, 256, 256, 1, P, 256, P, P, ws, None) == -2          # transposed rows % 16
+    assert q(P, 256, 256, 256, 1, P, 248, P, P, ws, None) == -2          # transposed row shorter than rows
+    assert q(P, 256, 256, 256, 2, P, 256, P, P, ws, None) == -8          # transpose flag
+    assert q(P, 256, 256, 256, 0, P, 256, P, P, 16, None) == -5          # workspace too small
+    assert q(P, 256, 256, 256, 0, None, 256, P, P, ws, None) == -1
+    assert q(P + 8, 256, 256, 256, 0, P, 256, P, P, ws, None) == -3
+    assert q(None, 0, 256, 256, 0, None, 256, None, None, 0, None) == 0   # empty tensor
+    a = so.attention_fp8
+    c = __import__("ctypes").c_float(0.0884)
+    #        Q  K  Vt B  S    H  ldq  ldk  ldvt sq sk sv scale O  ldo  stream
+    assert a(P, P, P, 1, 200, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -2     # S % 128
+    assert a(P, P, P, 1, 256, 2, 128, 256, 256, P, P, P, c, P, 256, None) == -2     # ldq < heads * 128
+    assert a(P, P, P, 2, 256, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -2     # ldvt < batch * S
+    assert a(P, P, P, 1, 256, 2, 256, 256, 256, P, P, P, __import__("ctypes").c_float(0.0), P, 256, None) == -8
+    assert a(P, P, P, 1, 256, 2, 256, 256, 256, None, P, P, c, P, 256, None) == -1
+    assert a(P, P, P + 4, 1, 256, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -3
+    assert a(None, None, None, 0, 256, 2, 256, 256, 0, None, None, None, c, None, 256, None) == 0
+    if not __import__("torch").cuda.is_available():
+        assert a(P, P, P, 1, 256, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -4   # valid: reaches the device check
+
+
 def test_quantize_next_argument_checks(so):
     """w4a4_gemm_quantize_next rejects bad column ranges, strides and pointers on the host."""
     P = 1 << 20
