@@ -819,6 +819,36 @@ def run_table(args):
     del pu, pd, X, qa_u, ws_u, H, ws_d, qa_d, Yd
     torch.cuda.empty_cache()
 
+    # FP8 attention on the sequences of the two block sizes (heads of 128):
+    # the three per-tensor E4M3 quantisations and the attention kernel
+    for S, H, what in ((4608, 24, "1024px sequence, hidden 3072"), (16896, 48, "2048px sequence, hidden 6144")):
+        ga = torch.Generator(device=dev)
+        ga.manual_seed(9000 + S)
+        q = (1.5 * torch.randn(S, H * 128, generator=ga, device=dev)).to(torch.bfloat16)
+        k = (1.5 * torch.randn(S, H * 128, generator=ga, device=dev)).to(torch.bfloat16)
+        v = torch.randn(S, H * 128, generator=ga, device=dev).to(torch.bfloat16)
+        tq, tk, tv = w4.quantize_fp8(q), w4.quantize_fp8(k), w4.quantize_fp8(v, transpose=True)
+        Oa = torch.empty(S, H * 128, dtype=torch.bfloat16, device=dev)
+        wsq = torch.empty(w4.fp8_quant_workspace_bytes(S, H * 128), dtype=torch.uint8, device=dev)
+
+        def quant3():
+            for x, t, tr in ((q, tq, False), (k, tk, False), (v, tv, True)):
+                w4.fp8_quantize(x, S, H * 128, H * 128, tr, t.codes, t.codes.stride(0), t.scale, wsq)
+
+        def att():
+            w4.attention(tq, tk, tv, H, O=Oa)
+        t_q, t_a = med_us([quant3, att])
+        check()
+        fl = 4.0 * S * S * 128 * H
+        qbytes = 3 * (2 * S * H * 128 + 2 * S * H * 128 + S * H * 128)   # amax read, quantise read, codes
+        emit({"table": "attention_fp8", "sequence": what, "S": S, "heads": H, "d_head": 128,
+              "attention_us": round(t_a, 1), "attention_tflops": tf(fl, t_a),
+              "attention_frac_fp8": round(tf(fl, t_a) / (peaks["bf16_tflops"] * 2.0), 3),
+              "fp8_peak_basis": "measured bf16 burst x 2 (nominal FP8/BF16)",
+              "quantise_qkv_us": round(t_q, 1), "quantise_qkv_gbs": round(qbytes / (t_q * 1e-6) / 1e9, 1)})
+        del q, k, v, tq, tk, tv, Oa, wsq
+        torch.cuda.empty_cache()
+
     # config 5: the denoising block (fused QKV + MLP-up projection on one
     # quantised activation, GELU on the MLP part, MLP-down) per step, and a
     # 50-step trajectory; every step re-quantises a fresh activation
@@ -894,6 +924,7 @@ CASES = {
     "quant_fused_flux1024": ("nvfp4_quantize_act, single pass (4608 x 3072)", 4608, 3072, None, None),
     "quant_two_pass_block2048": ("nvfp4_quantize_act, two passes (16896 x 6144)", 16896, 6144, None, None),
     "quant_stream_block2048": ("nvfp4_quantize_act_with_amax, streaming pass (16896 x 6144)", 16896, 6144, None, None),
+    "attention_fp8_small": ("attention_fp8 on 4096 tokens, 8 heads of 128 (E4M3 operands)", 4096, 1024, None, None),
     "pack_weight_block2048_out": ("nvfp4_pack_weight on an fp32 residual (6144 x 24576)", 6144, 24576, None, None),
 }
 
@@ -917,7 +948,17 @@ def run_case(args):
     inv_s = (1.0 / torch.exp(0.3 * torch.randn(K, generator=g, device=dev))).contiguous()
     L1t = (0.02 * torch.randn(r, K, generator=g, device=dev)).to(torch.bfloat16)
     t_w = torch.full((1,), 0.01, device=dev)
-    if args.case.startswith("pack_weight"):
+    if args.case.startswith("attention"):
+        heads = K // 128
+        tq = w4.quantize_fp8((1.5 * torch.randn(M, K, generator=g, device=dev)).to(torch.bfloat16))
+        tk = w4.quantize_fp8((1.5 * torch.randn(M, K, generator=g, device=dev)).to(torch.bfloat16))
+        tv = w4.quantize_fp8(torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16), transpose=True)
+        Oa = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+
+        def call():
+            w4.attention_fp8(tq.codes, tk.codes, tv.codes, 1, M, heads, K, K, M, tq.scale, tk.scale, tv.scale,
+                             1.0 / 128 ** 0.5, Oa, K, st)
+    elif args.case.startswith("pack_weight"):
         R = 0.02 * torch.randn(M, K, generator=g, device=dev)
         ws = w4.new_workspace(w4.nvfp4_quant_workspace_bytes(M, K, 0), dev)
         Wq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)

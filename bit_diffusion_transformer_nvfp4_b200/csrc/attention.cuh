@@ -10,7 +10,7 @@
 //   P = 2^(c S - m)      online softmax in fp32 (c = scale s_q s_k log2 e),
 //                        rounded to E4M3 for the second product
 //   O = sum_j P_j V_j    tcgen05.mma kind::f8f6f4 into a second TMEM accumulator
-// and writes bf16 O s_v / l (l = the sum of the rounded P).  The running
+// and writes bf16 O s_v / l (l = the sum of P before the rounding).  The running
 // offset m moves only when a tile's maximum exceeds it by more than half a
 // binade, and sits 8 binades above the largest probability so that E4M3's
 // range holds P from 2^-17 to 2^8.5 of the row's largest weight; O and l are
@@ -19,7 +19,9 @@
 // Roles (192 threads, two CTAs per SM): warp 0 TMA producer (the query tile
 // once, then key and value tiles through a two-stage ring), warp 1 TMEM owner
 // and the single MMA-issuing thread, warps 2-5 softmax (one query row per
-// thread: TMEM lane quarter warp % 4).
+// thread: TMEM lane quarter warp % 4).  A softmax thread copies its row's 128
+// scores into registers at once, so the next tile's Q K^T runs on the tensor
+// cores while this tile's probabilities are computed.
 #pragma once
 
 #include "sm100.cuh"
@@ -71,6 +73,38 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d, uint64_t adesc, uint64_t bd
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Blackwell packed fp32 fused multiply-add and add: two IEEE round-to-nearest results.
+__device__ __forceinline__ void fma2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                        float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Each thread of the warp reads 16 consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
 // Each thread of the warp writes 32 consecutive 32-bit columns of its lane.
@@ -167,20 +201,28 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_fp8_kernel(const __grid_
     if (lane == 0) {
       const uint32_t idesc = idesc_e4m3(kAttnTile, kAttnTile);
       const uint32_t q_base = smem_u32(smem + L::kQOff), p_base = smem_u32(smem + L::kPOff);
-      bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.status);
-      for (int j = 0; j < n_kv && ok; ++j) {
+      // S = Q K_j^T for tile j once its keys have landed and the softmax
+      // warps hold tile j-1's scores in registers
+      auto issue_s = [&](int j) -> bool {
         const int s = j % kAttnStages;
-        const uint32_t k_base = smem_u32(smem + L::kKOff + s * L::kStageBytes);
-        const uint32_t v_base = k_base + L::kTileBytes;
-        ok = mbar_wait(smem_u32(&kv_full[s]), (j / kAttnStages) & 1, abort_flag, p.status) &&
-             (j == 0 || mbar_wait(smem_u32(s_free), (j - 1) & 1, abort_flag, p.status));
-        if (!ok) break;
+        if (!mbar_wait(smem_u32(&kv_full[s]), (j / kAttnStages) & 1, abort_flag, p.status) ||
+            (j > 0 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, abort_flag, p.status)))
+          return false;
         tc_fence_after();
+        const uint32_t k_base = smem_u32(smem + L::kKOff + s * L::kStageBytes);
 #pragma unroll
         for (int k = 0; k < kAttnD / 32; ++k)
           mma_e4m3(t_s, smem_desc(q_base + 32 * k, 16, 1024, kSwizzle128B),
                    smem_desc(k_base + 32 * k, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
         tc_commit(smem_u32(s_full));
+        return true;
+      };
+      bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.status) && (n_kv == 0 || issue_s(0));
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j % kAttnStages;
+        const uint32_t v_base = smem_u32(smem + L::kKOff + s * L::kStageBytes) + L::kTileBytes;
+        // the next tile's scores overlap this tile's softmax
+        if (j + 1 < n_kv && !issue_s(j + 1)) break;
         if (!mbar_wait(smem_u32(p_full), j & 1, abort_flag, p.status)) break;
         tc_fence_after();
 #pragma unroll
@@ -211,17 +253,20 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_fp8_kernel(const __grid_
         break;
       }
       tc_fence_after();
-      // pass 1: the tile's row maximum
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < kAttnTile / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32cols(t_s + lane_base + 32 * cc, v);
-        tmem_ld_wait();
+      // the row's 128 scores into registers, and S's TMEM columns free for
+      // the next tile's Q K^T while this one's softmax runs
+      uint32_t sv[kAttnTile];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
-      }
-      const float m_tile = mx * c;
+      for (int cc = 0; cc < kAttnTile / 32; ++cc)
+        tmem_ld_32cols(t_s + lane_base + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(s_free));
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < kAttnTile; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(sv[i]));
+      const float m_tile = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;
       // the previous tile's P V products must be done before P is rewritten
       // or O is read
       if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(o_done), (j - 1) & 1, abort_flag, p.status))) {
@@ -236,37 +281,39 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_fp8_kernel(const __grid_
       const float f = (j > 0 && moves) ? ex2_approx(m_used - m_new) : 1.0f;
       if (__any_sync(0xffffffffu, j > 0 && moves)) {
         l *= f;
+        // 16 columns at a time: the row's scores stay in registers meanwhile
 #pragma unroll 1
-        for (int cc = 0; cc < kAttnD / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld_32cols(t_o + lane_base + 32 * cc, v);
+        for (int cc = 0; cc < kAttnD / 16; ++cc) {
+          uint32_t v[16];
+          tmem_ld_16cols(t_o + lane_base + 16 * cc, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-          tmem_st_32cols(t_o + lane_base + 32 * cc, v);
+          for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+          tmem_st_16cols(t_o + lane_base + 16 * cc, v);
         }
         tmem_st_wait();
       }
       m_used = m_new;
       const float off = m_used - kAttnOffset;
-      // pass 2: P = 2^(c s - off) in E4M3, 32 keys at a time, into the row
-      // of the swizzled P tile; l sums the rounded values
-#pragma unroll 1
+      // P = 2^(c s - off) in E4M3, 32 keys at a time, into the row of the
+      // swizzled P tile; l sums the probabilities (the rounding to E4M3 is
+      // unbiased, so the sum of the rounded ones differs from it far less
+      // than each product does)
+      float la = 0.0f, lb = 0.0f;
+#pragma unroll
       for (int cc = 0; cc < kAttnTile / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32cols(t_s + lane_base + 32 * cc, v);
-        tmem_ld_wait();
         uint32_t b[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float p0 = ex2_approx(__fmaf_rn(__uint_as_float(v[4 * i]), c, -off));
-          const float p1 = ex2_approx(__fmaf_rn(__uint_as_float(v[4 * i + 1]), c, -off));
-          const float p2 = ex2_approx(__fmaf_rn(__uint_as_float(v[4 * i + 2]), c, -off));
-          const float p3 = ex2_approx(__fmaf_rn(__uint_as_float(v[4 * i + 3]), c, -off));
-          const uint32_t lo = cvt_e4m3x2(p1, p0), hi = cvt_e4m3x2(p3, p2);
-          b[i] = lo | (hi << 16);
-          const float2 d0 = e4m3x2_to_f32(lo), d1 = e4m3x2_to_f32(hi);
-          l += (d0.x + d0.y) + (d1.x + d1.y);
+          const uint32_t* v = &sv[32 * cc + 4 * i];
+          float x0, x1, x2, x3;
+          fma2_rn(x0, x1, __uint_as_float(v[0]), __uint_as_float(v[1]), c, c, -off, -off);
+          fma2_rn(x2, x3, __uint_as_float(v[2]), __uint_as_float(v[3]), c, c, -off, -off);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+          b[i] = cvt_e4m3x2(p1, p0) | (cvt_e4m3x2(p3, p2) << 16);
+          float s0, s1;
+          add2_rn(s0, s1, p0, p1, p2, p3);
+          add2_rn(la, lb, la, lb, s0, s1);
         }
         // keys 32cc .. 32cc+31: 16-byte units 2cc and 2cc+1 of the row
 #pragma unroll
@@ -274,13 +321,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_fp8_kernel(const __grid_
           *reinterpret_cast<uint4*>(prow + (((2 * cc + u) ^ (r & 7)) << 4)) =
               make_uint4(b[4 * u], b[4 * u + 1], b[4 * u + 2], b[4 * u + 3]);
       }
-      tc_fence_before();
+      l += la + lb;
       fence_proxy_async_smem();  // P written by this thread, read by the tensor core
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(s_free));
-        mbar_arrive(smem_u32(p_full));
-      }
+      if (lane == 0) mbar_arrive(smem_u32(p_full));
     }
     if (ok && n_kv > 0 && __all_sync(0xffffffffu, mbar_wait(smem_u32(o_done), (n_kv - 1) & 1, abort_flag, p.status))) {
       tc_fence_after();

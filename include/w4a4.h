@@ -389,7 +389,9 @@ int fp8_quantize(const void* X, int64_t rows, int64_t cols, int64_t ldx, int tra
  * The kernel computes S = Q K^T on the tensor cores in fp32, an online
  * softmax in fp32 with the probabilities rounded to E4M3 (within 2^-17 to
  * 2^8.5 of the row's running maximum) for the second product O += P V, and
- * writes bf16(O s_v / l), l the sum of the rounded probabilities.  One CTA
+ * writes bf16(O s_v / l), l the sum of the probabilities before their
+ * rounding (unbiased, so it differs from the sum of the rounded ones far
+ * less than the rounding changes each product).  One CTA
  * per (128 queries, head, sequence), two per SM; programmatic stream
  * serialisation as for the GEMMs.
  */
