@@ -1034,6 +1034,49 @@ def run_case(args):
         raise RuntimeError(f"device status {status}")
 
 
+def run_fp4_peak(args):
+    """The measured FP4 peak: w4a4_fp4_mma_rate on every SM, CTA pairs
+    (256 x 256 x 64 MMAs) and single CTAs (128 x 256 x 64), --fp4-iters MMAs
+    per issuer, event-timed launches after warm-up ones; the issuers' own
+    cycle counts give the clock.  One JSON line per mode."""
+    import torch
+    import bit_diffusion_transformer_nvfp4_b200 as w4
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w4.lib()
+    st = torch.cuda.current_stream()
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    cycles = torch.zeros(n_sm, dtype=torch.int64, device=dev)
+    peaks, peak_kind = load_peaks()
+    for pair in (1, 0):
+        issuers = n_sm // 2 if pair else n_sm
+        flops = 2.0 * (256 if pair else 128) * 256 * 64
+        for _ in range(max(args.warmup, 3)):
+            w4.w4a4_fp4_mma_rate(args.fp4_iters, pair, cycles, st)
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            w4.w4a4_fp4_mma_rate(args.fp4_iters, pair, cycles, st)
+            e1.record(st)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        status = w4.w4a4_device_status()
+        c = cycles[:issuers].cpu().numpy().astype(np.float64)
+        t = statistics.median(ms)
+        tflops = issuers * args.fp4_iters * flops / (t * 1e-3) / 1e12
+        print(json.dumps({"fp4_mma_rate": "pair 256x256x64" if pair else "single 128x256x64",
+                          "issuers": issuers, "mmas_per_issuer": args.fp4_iters, "ms": round(t, 4),
+                          "tflops": round(tflops, 1),
+                          "cycles_per_mma": round(float(np.median(c)) / args.fp4_iters, 2),
+                          "sm_mhz_from_cycles": round(float(np.median(c)) / (t * 1e-3) / 1e6, 1),
+                          "vs_nominal_fp4_of_measured_bf16": round(tflops / (peaks["bf16_tflops"] * FP4_OVER_BF16), 3),
+                          "status": status}), flush=True)
+        if status != 0 or not np.all(c > 0):
+            raise RuntimeError(f"device status {status}")
+
+
 # ---------------------------------------------------------------- oracle arms
 
 def cpu_threads():
@@ -1146,10 +1189,15 @@ def main():
     ap.add_argument("--table-reps", type=int, default=20)
     ap.add_argument("--case", choices=sorted(CASES),
                     help="run one kernel's small profiling workload (--steps calls after --warmup) instead")
+    ap.add_argument("--fp4-peak", action="store_true",
+                    help="measure the FP4 tensor-core instruction rate (back-to-back MMAs on every SM) instead")
+    ap.add_argument("--fp4-iters", type=int, default=100000)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.case:
+    if args.fp4_peak:
+        run_fp4_peak(args)
+    elif args.case:
         run_case(args)
     elif args.table:
         run_table(args)

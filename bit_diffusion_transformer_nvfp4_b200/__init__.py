@@ -26,6 +26,7 @@ __all__ = [
     "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
     "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next", "w4a4_gemm_rope", "gemm_rope",
     "fp8_quant_workspace_bytes", "fp8_quantize", "attention_fp8", "Fp8Tensor", "quantize_fp8", "attention",
+    "w4a4_fp4_mma_rate",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -55,6 +56,7 @@ _SIG = {
     "w4a4_gemm_rope": (_c.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _c.c_int, _P, _I64, _I64, _P,
                                   _I64, _I64, _P, _I64, _P, _I64, _P, _P, _P]),
     "fp8_quant_workspace_bytes": (_c.c_size_t, [_I64, _I64]),
+    "w4a4_fp4_mma_rate": (_c.c_int, [_c.c_int, _c.c_int, _P, _P]),
     "fp8_quantize": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_int, _P, _I64, _P, _P, _c.c_size_t, _P]),
     "attention_fp8": (_c.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _c.c_float, _P, _I64,
                                  _P]),
@@ -179,6 +181,10 @@ def w4a4_gemm_rope(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_rope,
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), n_rope, d_head, _ptr(rope), ld_rope, n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s),
         _ptr(next_amax), _stream(stream)))
+
+
+def w4a4_fp4_mma_rate(iters, pair, cycles, stream=None):
+    _check("w4a4_fp4_mma_rate", lib().w4a4_fp4_mma_rate(int(iters), int(pair), _ptr(cycles), _stream(stream)))
 
 
 def fp8_quant_workspace_bytes(rows, cols) -> int:

@@ -18,6 +18,7 @@
 
 #include "quant.cuh"
 #include "attention.cuh"
+#include "mma_rate.cuh"
 
 namespace w4a4 {
 
@@ -91,6 +92,10 @@ int device_setup(DeviceInfo** out) {
                                   FusedQuantSmem::kBytes) == cudaSuccess;
   attr_ok &= cudaFuncSetAttribute(attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::kBytes) ==
              cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(fp4_mma_rate_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kRateSmem) == cudaSuccess;
+  attr_ok &= cudaFuncSetAttribute(fp4_mma_rate_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kRateSmem) == cudaSuccess;
   using G256 = GemmCfg<256, 4>;
   using G192 = GemmCfg<192, 4>;
 
@@ -964,6 +969,35 @@ int attention_fp8(const uint8_t* Q8, const uint8_t* K8, const uint8_t* Vt8, int6
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, attn_fp8_kernel, tq, tk, tv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  return W4A4_OK;
+}
+
+int w4a4_fp4_mma_rate(int iters, int pair, unsigned long long* cycles, void* stream) {
+  if (iters < 1 || iters > (1 << 20)) return W4A4_ERR_SHAPE;
+  if (pair != 0 && pair != 1) return W4A4_ERR_ARG;
+  if (!cycles) return W4A4_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(cycles) % 8 != 0) return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  int st = device_setup(&dev);
+  if (st != W4A4_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pair ? 2 * (dev->num_sms / 2) : dev->num_sms), 1, 1);
+  cfg.blockDim = dim3(kRateThreads, 1, 1);
+  cfg.dynamicSmemBytes = kRateSmem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pair ? 1 : 0;
+  const cudaError_t e = pair ? cudaLaunchKernelEx(&cfg, fp4_mma_rate_kernel<true>, iters, cycles, dev->status_ptr)
+                             : cudaLaunchKernelEx(&cfg, fp4_mma_rate_kernel<false>, iters, cycles, dev->status_ptr);
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return W4A4_ERR_CUDA;
   }

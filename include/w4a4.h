@@ -401,6 +401,24 @@ int attention_fp8(const uint8_t* Q8, const uint8_t* K8, const uint8_t* Vt8, int6
                   void* stream);
 
 /*
+ * w4a4_fp4_mma_rate -- a measurement, not part of the layer: the rate of the
+ * block-scaled FP4 tensor-core instruction the GEMM is built on
+ * (tcgen05.mma kind::mxf4nvf4.block_scale.block16), issued back to back with
+ * resident operands (pseudo-random codes, scale bytes 0x30..0x3F) on every
+ * SM.  It gives the measured FP4 peak beside the nominal one; the pages quote
+ * the FP4 tensor-core speedup only as a ratio ("Four Bits ...": 4x over FP16).
+ *   iters   MMAs per issuing thread, 1 .. 2^20
+ *   pair    1: 256 x 256 x 64 MMAs on CTA pairs (cta_group::2, one issuer per
+ *           two SMs); 0: 128 x 256 x 64 MMAs, one CTA and issuer per SM
+ *   cycles  out: device array of at least (number of SMs) entries; entry i is
+ *           the SM clock cycles issuer i took for its MMAs, from its first
+ *           issue to the completion of its last (0 if its wait gave up)
+ * One kernel on `stream`; time it with events to get the rate in FLOP/s
+ * (2 * 256 * 256 * 64 or 2 * 128 * 256 * 64 FLOPs per MMA).
+ */
+int w4a4_fp4_mma_rate(int iters, int pair, unsigned long long* cycles, void* stream);
+
+/*
  * w4a4_linear -- the whole hot path: nvfp4_quantize_act on X (row stride K)
  * into the workspace, then w4a4_gemm into Y (row stride N).
  *   workspace >= w4a4_workspace_bytes(M, N, K, r) bytes of device memory.

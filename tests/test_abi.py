@@ -260,6 +260,19 @@ def test_fp8_argument_checks(so):
         assert a(P, P, P, 1, 256, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -4   # valid: reaches the device check
 
 
+def test_fp4_mma_rate_argument_checks(so):
+    """w4a4_fp4_mma_rate rejects bad counts, modes and pointers on the host."""
+    P = 1 << 20
+    f = so.w4a4_fp4_mma_rate
+    assert f(0, 1, P, None) == -2
+    assert f((1 << 20) + 1, 1, P, None) == -2
+    assert f(100, 2, P, None) == -8
+    assert f(100, 1, None, None) == -1
+    assert f(100, 0, P + 4, None) == -3
+    if not __import__("torch").cuda.is_available():
+        assert f(100, 1, P, None) == -4        # valid: reaches the device check
+
+
 def test_quantize_next_argument_checks(so):
     """w4a4_gemm_quantize_next rejects bad column ranges, strides and pointers on the host."""
     P = 1 << 20
