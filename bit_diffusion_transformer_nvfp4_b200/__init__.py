@@ -26,7 +26,7 @@ __all__ = [
     "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
     "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next", "w4a4_gemm_rope", "gemm_rope",
     "fp8_quant_workspace_bytes", "fp8_quantize", "attention_fp8", "Fp8Tensor", "quantize_fp8", "attention",
-    "w4a4_fp4_mma_rate",
+    "w4a4_fp4_mma_rate", "w4a4_last_error",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -67,6 +67,7 @@ _SIG = {
                                _P, _c.c_size_t, _P]),
     "nvfp4_quantize_act_noalloc": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _c.c_int, _P, _P, _P, _P, _P, _P]),
     "w4a4_device_status": (_c.c_int, [_c.POINTER(_c.c_int), _c.c_int]),
+    "w4a4_last_error": (_c.c_int, []),
     "w4a4_set_wait_bound": (_c.c_int, [_I64]),
     "nvfp4_sf_to_rowmajor": (_c.c_int, [_P, _I64, _I64, _P, _P]),
     "w4a4_status_string": (_c.c_char_p, [_c.c_int]),
@@ -181,6 +182,12 @@ def w4a4_gemm_rope(Xq, Xsf, t_x, U, M, N, K, Wq, Wsf, t_w, L2t, r, bias, n_rope,
         _ptr(Xq), _ptr(Xsf), _ptr(t_x), _ptr(U), M, N, K, _ptr(Wq), _ptr(Wsf), _ptr(t_w), _ptr(L2t), r,
         _ptr(bias), n_rope, d_head, _ptr(rope), ld_rope, n_plain, _ptr(Y), ldy, _ptr(H), ldh, _ptr(next_inv_s),
         _ptr(next_amax), _stream(stream)))
+
+
+def w4a4_last_error() -> int:
+    """The sticky device status (no device synchronisation: synchronise the
+    streams of interest first)."""
+    return lib().w4a4_last_error()
 
 
 def w4a4_fp4_mma_rate(iters, pair, cycles, stream=None):

@@ -1141,6 +1141,32 @@ int w4a4_device_status(int* status, int reset) {
   return W4A4_OK;
 }
 
+int w4a4_last_error(void) {
+  // the sticky status word as it stands, read on a private non-blocking
+  // stream: no wait for the caller's work (the caller synchronises first)
+  static cudaStream_t reader[kMaxDevices] = {};
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!reader[d] && cudaStreamCreateWithFlags(&reader[d], cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      reader[d] = nullptr;
+      return W4A4_ERR_CUDA;
+    }
+  }
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, reader[d]) != cudaSuccess ||
+      cudaStreamSynchronize(reader[d]) != cudaSuccess) {
+    cudaGetLastError();
+    return W4A4_ERR_CUDA;
+  }
+  return v;
+}
+
 int w4a4_set_wait_bound(int64_t cycles) {
   if (cycles <= 0) cycles = kDefaultWaitBoundCycles;
   if (cycles < 1000000) return W4A4_ERR_ARG;

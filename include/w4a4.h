@@ -476,6 +476,15 @@ int nvfp4_quantize_act_noalloc(const void* X, int64_t M, int64_t K, int64_t ldx,
  * or W4A4_ERR_CUDA. */
 int w4a4_device_status(int* status, int reset);
 
+/*
+ * w4a4_last_error -- the sticky device status word of the current device
+ * (W4A4_OK, W4A4_ERR_DEVICE_TIMEOUT or W4A4_ERR_DEVICE_LAYOUT), read without
+ * synchronising the device: call it after synchronising the streams whose
+ * work it should cover.  Does not clear the word (w4a4_device_status with
+ * reset does).  W4A4_ERR_CUDA if the read itself fails.
+ */
+int w4a4_last_error(void);
+
 /* Sets how long a device-side wait (pipeline barrier, grid barrier, counter)
  * spins before it gives up, records W4A4_ERR_DEVICE_TIMEOUT in the sticky
  * status word, drains its own copies and returns: ``cycles`` SM clock cycles

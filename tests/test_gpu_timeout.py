@@ -42,7 +42,10 @@ def test_wait_runs_out_and_the_library_recovers():
     try:
         w4.quantize_act(X, inv_s, L1t, t_w, workspace=ws)
         torch.cuda.synchronize()                          # the kernel ended on its own
+        assert w4.w4a4_last_error() == TIMEOUT_STATUS     # read without a device synchronisation
+        assert w4.w4a4_last_error() == TIMEOUT_STATUS     # sticky: reading does not clear it
         assert w4.w4a4_device_status(reset=True) == TIMEOUT_STATUS
+        assert w4.w4a4_last_error() == 0
     finally:
         w4.w4a4_set_wait_bound(0)
     assert w4.w4a4_device_status() == 0
