@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kRateThreads, 1) fp4_mma_rate_kernel(int iters
   uint64_t* done = reinterpret_cast<uint64_t*>(smem_raw + kRateABytes + kRateBBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
   // operands: pseudo-random code bytes
