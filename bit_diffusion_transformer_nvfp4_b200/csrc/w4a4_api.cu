@@ -921,8 +921,8 @@ int attention_fp8(const uint8_t* Q8, const uint8_t* K8, const uint8_t* Vt8, int6
                   int64_t ldq, int64_t ldk, int64_t ldvt, const float* s_q, const float* s_k, const float* s_v,
                   float softmax_scale, void* O, int64_t ldo, void* stream) {
   if (batch < 0 || S < 0 || heads <= 0 || S % kAttnTile != 0 || heads > 65535 || batch > 65535 ||
-      S > (int64_t(1) << 24))
-    return W4A4_ERR_SHAPE;
+      S > (int64_t(1) << 24) || batch * S > (int64_t(1) << 30) || heads * kAttnD > (int64_t(1) << 30))
+    return W4A4_ERR_SHAPE;  // (token and feature coordinates stay 32-bit)
   const int64_t width = heads * kAttnD;
   if (ldq < width || ldq % 16 != 0 || ldk < width || ldk % 16 != 0 || ldvt < batch * S || ldvt % 16 != 0 ||
       ldo < width || ldo % 8 != 0)

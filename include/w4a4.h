@@ -376,8 +376,8 @@ int fp8_quantize(const void* X, int64_t rows, int64_t cols, int64_t ldx, int tra
 
 /*
  * attention_fp8 -- O = softmax(c Q K^T) V per head and sequence, on E4M3
- * operands: batch sequences of S tokens (S % 128 == 0), heads of 128
- * features.
+ * operands: batch sequences of S tokens (S % 128 == 0, batch * S <= 2^30),
+ * heads of 128 features.
  *   Q8, K8  in  E4M3 [batch * S, ldq / ldk bytes], token-major, head h in
  *               columns h*128 .. h*128+127 (ld >= heads*128, ld % 16 == 0)
  *   Vt8     in  E4M3 [heads * 128, ldvt bytes]: V transposed, row h*128 + d,

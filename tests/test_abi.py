@@ -250,6 +250,7 @@ def test_fp8_argument_checks(so):
     c = __import__("ctypes").c_float(0.0884)
     #        Q  K  Vt B  S    H  ldq  ldk  ldvt sq sk sv scale O  ldo  stream
     assert a(P, P, P, 1, 200, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -2     # S % 128
+    assert a(P, P, P, 1 << 8, 1 << 23, 1, 128, 128, 1 << 31, P, P, P, c, P, 128, None) == -2   # tokens beyond 2^30
     assert a(P, P, P, 1, 256, 2, 128, 256, 256, P, P, P, c, P, 256, None) == -2     # ldq < heads * 128
     assert a(P, P, P, 2, 256, 2, 256, 256, 256, P, P, P, c, P, 256, None) == -2     # ldvt < batch * S
     assert a(P, P, P, 1, 256, 2, 256, 256, 256, P, P, P, __import__("ctypes").c_float(0.0), P, 256, None) == -8
