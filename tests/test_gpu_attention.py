@@ -69,7 +69,7 @@ def run(w4, q, k, v, heads, batch):
     return from_dev_bf16(O), ref
 
 
-@pytest.mark.parametrize("batch,S,heads", [(1, 256, 2), (2, 384, 3), (1, 1024, 1)])
+@pytest.mark.parametrize("batch,S,heads", [(1, 256, 2), (2, 384, 3), (1, 1024, 1), (3, 128, 2)])
 def test_attention_random(w4, batch, S, heads):
     g = rng(100 * batch + S + heads)
     M = batch * S
