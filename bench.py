@@ -11,13 +11,16 @@ up-projection and the bf16 cast.  Inputs are synthetic and seeded (per-channel
 lognormal(0, 1.5) activation magnitudes, N(0, 0.02) weights), drawn on the GPU.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload block2048|qkv1024] [--table]
+                    [--workload block2048|qkv1024] [--table] [--case NAME] [--fp4-peak]
 
 Prints one JSON line.  Under torchrun (N > 1) every rank runs an independent
 replica on its own GPU (the path has no cross-GPU exchange); rank 0 prints.
 ``--impl reference`` times the plain CPU oracle on the host cores instead.
 ``--workload qkv1024`` runs the FLUX-1024px QKV projection instead (M = 4608,
-3072 -> 9216); ``--table`` times every configuration's layers.
+3072 -> 9216); ``--table`` times every configuration's layers (with the
+SwiGLU, rotary and quantising epilogues and FP8 attention); ``--case`` runs
+one kernel's small workload for a profiler; ``--fp4-peak`` measures the FP4
+tensor-core instruction rate.
 """
 from __future__ import annotations
 
