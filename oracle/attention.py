@@ -46,10 +46,14 @@ def fp8_scale(amax) -> np.float32:
     return s
 
 
-def fp8_quantize(x: np.ndarray):
-    """x (bf16 values as fp32) -> (E4M3 codes, per-tensor scale s)."""
+def fp8_quantize(x: np.ndarray, amax=None):
+    """x (bf16 values as fp32) -> (E4M3 codes, per-tensor scale s).  ``amax``
+    gives the whole tensor's maximum magnitude when x is a part of it (every
+    element is coded on its own once the scale is fixed)."""
     x = np.asarray(x, dtype=np.float32)
-    s = fp8_scale(np.max(np.abs(x)) if x.size else F32(0.0))
+    if amax is None:
+        amax = np.max(np.abs(x)) if x.size else F32(0.0)
+    s = fp8_scale(amax)
     inv = F32(F32(1.0) / s)
     codes = e4m3_encode((x * inv).astype(np.float32))
     return codes, s

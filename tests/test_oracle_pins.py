@@ -553,6 +553,14 @@ def test_fp8_tensor_quantiser():
     assert np.all(np.abs(back - x) <= np.abs(x) * 2.0 ** -4 + float(s) * 2.0 ** -10)   # half an E4M3 step
     z, s0 = attention.fp8_quantize(np.zeros((3, 4), np.float32))
     assert s0 == 1.0 and not np.any(z)
+    # a part of the tensor under the whole tensor's amax: the same scale and
+    # the same bytes as those elements of the whole tensor's coding
+    rest = np.delete(np.arange(64), i[0])[:6]                     # rows without the maximum
+    part, sp = attention.fp8_quantize(x[rest, 10:30], amax=np.max(np.abs(x)))
+    assert sp == s
+    np.testing.assert_array_equal(part, codes[rest, 10:30])
+    own, so = attention.fp8_quantize(x[rest, 10:30])
+    assert so < s and np.any(own != part)                        # its own amax is smaller: other codes
 
 
 def test_attention_two_keys_by_hand():
