@@ -114,3 +114,46 @@ def test_attention_dominant_key(w4):
     np.testing.assert_allclose(o[sel], ref[sel], rtol=2.0 ** -7, atol=2.0 ** -7 * np.max(np.abs(v)))
     rest = np.arange(128, S)                              # the others: every score 0, O = mean of V
     assert olinear.rel_frobenius(o[rest], ref[rest]) <= 4e-3
+
+
+@pytest.mark.parametrize("S,heads", [(4608, 24), (16896, 48)])
+def test_attention_full_size_sampled(w4, S, heads):
+    """The sequences of the two block sizes (1024px: 4608 tokens, 24 heads;
+    2048px: 16896 tokens, 48 heads), one sequence, in the launch the
+    benchmark table times.  Every scale against the oracle's; the codes of
+    sampled heads (all keys and values, sampled query rows) byte for byte
+    under the whole tensor's amax; O of those rows and heads against the
+    oracle's exact attention over all S keys."""
+    import torch
+    g = rng(9100 + S)
+    D = heads * 128
+    q = bf16_round(g.standard_normal((S, D), np.float32) * np.float32(1.5))
+    k = bf16_round(g.standard_normal((S, D), np.float32) * np.float32(1.5))
+    v = bf16_round(g.standard_normal((S, D), np.float32))
+    tq = w4.quantize_fp8(to_dev_bf16(q))
+    tk = w4.quantize_fp8(to_dev_bf16(k))
+    tv = w4.quantize_fp8(to_dev_bf16(v), transpose=True)
+    O = w4.attention(tq, tk, tv, heads)
+    torch.cuda.synchronize()
+    assert w4.w4a4_device_status() == 0
+    amax = [np.max(np.abs(a)) for a in (q, k, v)]
+    for t, a in zip((tq, tk, tv), amax):
+        assert float(t.scale.cpu()[0]) == float(oatt.fp8_scale(a))
+    rows = np.sort(g.choice(S, 40, replace=False))
+    rows[0], rows[-1] = 0, S - 1
+    o_rows = from_dev_bf16(O[torch.from_numpy(rows).cuda()])
+    q_rows = tq.codes[torch.from_numpy(rows).cuda()].cpu().numpy()
+    for h in (0, heads // 2 + 1, heads - 1):
+        cols = slice(h * 128, (h + 1) * 128)
+        cq, sq = oatt.fp8_quantize(q[rows, cols], amax=amax[0])
+        ck, sk = oatt.fp8_quantize(k[:, cols], amax=amax[1])
+        cv, sv = oatt.fp8_quantize(v[:, cols], amax=amax[2])
+        np.testing.assert_array_equal(q_rows[:, cols], cq)
+        np.testing.assert_array_equal(tk.codes[:, cols].cpu().numpy(), ck)
+        np.testing.assert_array_equal(tv.codes[cols].cpu().numpy(), cv.T)
+        ref = oatt.attention(oatt.fp8_dequantize(cq, sq), oatt.fp8_dequantize(ck, sk),
+                             oatt.fp8_dequantize(cv, sv), 1)
+        o = o_rows[:, cols]
+        assert np.all(np.isfinite(o))
+        rel = olinear.rel_frobenius(o, ref)
+        assert rel <= REL_FP8_P, f"head {h}: relative Frobenius error {rel:.3e}"
