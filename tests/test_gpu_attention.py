@@ -11,6 +11,9 @@
   2^8 exactly, so O is the mean of the values) and one dominant key per
   query (every other probability underflows, so O is that key's value) --
   both checked to the bf16 rounding of the output.
+* The full sequences of both block sizes (4608 tokens x 24 heads, 16896
+  tokens x 48 heads): scales, the codes of sampled heads and O of sampled
+  query rows against the oracle over all keys.
 """
 import numpy as np
 import pytest
