@@ -252,7 +252,16 @@ QuantPlan quant_plan(int64_t M, int64_t K, int r) {
   return q;
 }
 
-bool valid_k(int64_t K) { return K >= 64 && K % 64 == 0 && K <= (int64_t(1) << 30); }
+// Largest K: the tensor-amax pass gives every CTA kAmaxThreads 16-byte
+// column segments of a row and keeps at most kAmaxMaxBlocks partial maxima,
+// so a row spans at most kAmaxMaxBlocks x kAmaxThreads segments: 2^20 fp32
+// (weight) or 2^21 bf16 columns.  One bound for every entry point.
+constexpr int64_t kMaxK = int64_t(kAmaxMaxBlocks) * kAmaxThreads * 4;
+static_assert(kMaxK == (int64_t(1) << 20) && kMaxK == W4A4_MAX_K, "K bound of the header");
+// Largest column count of fp8_quantize (bf16 only: eight per segment).
+constexpr int64_t kFp8MaxCols = int64_t(kAmaxMaxBlocks) * kAmaxThreads * 8;
+
+bool valid_k(int64_t K) { return K >= 64 && K % 64 == 0 && K <= kMaxK; }
 
 // Rows the per-row-block low-rank counters of a workspace cover.
 bool valid_lowrank_rows(int64_t M, int r) { return r == 0 || M <= W4A4_MAX_LOWRANK_ROWS; }
@@ -864,7 +873,7 @@ int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* 
 }
 
 size_t fp8_quant_workspace_bytes(int64_t rows, int64_t cols) {
-  if (rows < 0 || cols <= 0 || cols % 8 != 0) return 0;
+  if (rows < 0 || cols <= 0 || cols % 8 != 0 || cols > kFp8MaxCols) return 0;
   return sizeof(float) * kAmaxMaxBlocks;  // the tensor-amax partial maxima
 }
 
@@ -872,7 +881,7 @@ int fp8_quantize(const void* X, int64_t rows, int64_t cols, int64_t ldx, int tra
                  float* scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (transpose != 0 && transpose != 1) return W4A4_ERR_ARG;
   if (rows < 0 || cols <= 0 || cols % 8 != 0 || ldx < cols || ldx % 8 != 0 || rows > (int64_t(1) << 30) ||
-      cols > (int64_t(1) << 30))
+      cols > kFp8MaxCols)
     return W4A4_ERR_SHAPE;
   if (transpose ? (rows % 16 != 0 || ldo < rows || ldo % 16 != 0) : (ldo < cols || ldo % 8 != 0))
     return W4A4_ERR_SHAPE;

@@ -47,8 +47,10 @@
  *     the legacy default stream).  Scalars (t_x, t_w) stay in device memory.
  *   - Host-detectable problems return an error before anything is enqueued.
  *   - Pointers must be 16-byte aligned; ldx/ldr/ldy are in elements.
- *   - Constraints: K % 64 == 0, K >= 64 (one FP4 MMA K-step of four 16-element
- *     scale blocks); N % 8 == 0; r in {0, 16, 32}
+ *   - Constraints: K % 64 == 0, 64 <= K <= W4A4_MAX_K (one FP4 MMA K-step of
+ *     four 16-element scale blocks; the bound is the widest row the
+ *     tensor-amax pass covers with its fixed count of partial maxima);
+ *     N % 8 == 0; r in {0, 16, 32}
  *     (rank 16 is the pages' choice for the low-rank branch, "SVDQuant
  *     Guide ...", "The Solution ..." and "Empirical Efficiency Benchmark");
  *     M >= 0, rows need not be a multiple of 128.  An empty problem (M == 0;
@@ -85,6 +87,9 @@ typedef enum {
   W4A4_ERR_SCRATCH_LIMIT = -9,  /* problem needs more than the built-in scratch (no-alloc entry) */
   W4A4_ERR_DEVICE_LAYOUT = -10  /* sticky device status: a kernel found its shared memory misaligned */
 } w4a4_status;
+
+/* Largest K (columns of an activation or weight) every entry point accepts. */
+#define W4A4_MAX_K ((int64_t)1 << 20)
 
 enum { W4A4_EPI_NONE = 0, W4A4_EPI_GELU_TANH = 1 };
 enum { W4A4_SRC_BF16 = 0, W4A4_SRC_F32 = 1 };
@@ -361,7 +366,7 @@ int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* 
  * (out[r * ldo + c], transpose = 0) or transposed (out[c * ldo + r],
  * transpose = 1: the value layout attention_fp8 reads).  Two kernels: the
  * tensor amax into the workspace, then the codes.
- *   cols % 8 == 0, ldx >= cols, ldx % 8 == 0; transpose: rows % 16 == 0,
+ *   cols % 8 == 0, cols <= 2^21, ldx >= cols, ldx % 8 == 0; transpose: rows % 16 == 0,
  *   ldo >= rows, ldo % 16 == 0; else ldo >= cols, ldo % 8 == 0
  *   scale     out fp32 device scalar (4-byte aligned)
  *   workspace >= fp8_quant_workspace_bytes(rows, cols) bytes of device memory

@@ -86,6 +86,27 @@ def test_host_validation_before_any_launch(so):
 
 
 
+def test_k_and_fp8_column_bounds(so):
+    """K up to 2^20 (the widest row the tensor-amax pass covers with its 1024
+    partial maxima of 256 segments) and FP8 columns up to 2^21 are accepted;
+    one step past either bound is a size error before any launch."""
+    P = 1 << 20
+    big = 1 << 30
+    kmax = 1 << 20
+    assert so.nvfp4_quant_workspace_bytes(128, kmax, 32) > 0
+    assert so.nvfp4_quant_workspace_bytes(128, kmax + 64, 32) == 0
+    assert so.w4a4_workspace_bytes(128, 256, kmax, 32) > 0
+    assert so.w4a4_workspace_bytes(128, 256, kmax + 64, 32) == 0
+    assert so.nvfp4_quantize_act(P, 128, kmax + 64, kmax + 64, None, None, 0, None, P, P, P, None, P, big,
+                                 None) == -2
+    assert so.nvfp4_pack_weight(P, 1, 128, kmax + 64, kmax + 64, P, P, P, P, big, None) == -2
+    assert so.w4a4_gemm(P, P, P, None, 128, 128, kmax + 64, P, P, P, None, 0, None, 0, P, 128, None) == -2
+    assert so.w4a4_linear(P, 128, 128, kmax + 64, P, P, P, None, P, P, 32, None, 0, P, P, big, None) == -2
+    assert so.fp8_quant_workspace_bytes(128, 1 << 21) > 0
+    assert so.fp8_quant_workspace_bytes(128, (1 << 21) + 8) == 0
+    assert so.fp8_quantize(P, 128, (1 << 21) + 8, (1 << 21) + 8, 0, P, (1 << 21) + 8, P, P, big, None) == -2
+
+
 def test_host_validation_linear_and_amax_entries(so):
     """The whole-path and given/next-amax entry points reject bad arguments on
     the host, in the documented order, before touching a GPU."""
