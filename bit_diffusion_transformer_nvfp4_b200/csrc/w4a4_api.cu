@@ -845,7 +845,7 @@ int w4a4_gemm_quantize_next(const uint8_t* Xq, const uint8_t* Xsf, const float* 
   if (swiglu && ((N - n_plain) % 32 != 0 || epilogue != W4A4_EPI_NONE)) return W4A4_ERR_SHAPE;
   const int64_t n_out = swiglu ? (N - n_plain) / 2 : N;  // the outputs quantised for the next layer
   if (n_out % 32 != 0 || next_K % 64 != 0 || next_col < 0 || next_col % 64 != 0 || next_col + n_out > next_K ||
-      next_ldq < next_K / 2 || next_ldq % 16 != 0 || next_K > (int64_t(1) << 30))
+      next_ldq < next_K / 2 || next_ldq % 16 != 0 || next_K > kMaxK)
     return W4A4_ERR_SHAPE;
   if (swiglu && H != nullptr && (ldh < n_out || ldh % 8 != 0)) return W4A4_ERR_SHAPE;
   if (n_plain > 0 && Y != nullptr && (ldy < n_plain || ldy % 8 != 0)) return W4A4_ERR_SHAPE;
@@ -1050,6 +1050,7 @@ int nvfp4_sf_to_rowmajor(const uint8_t* sf_atoms, int64_t rows, int64_t K, uint8
   if (st != W4A4_OK) return st;
   const int64_t n = rows * (K / kQChunk);
   const int64_t blocks = ceil_div(n, 256);
+  if (blocks > INT32_MAX) return W4A4_ERR_SHAPE;  // one grid dimension
   sf_to_rowmajor_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       sf_atoms, rows, K / kQChunk, sf_rowmajor);
   if (cudaGetLastError() != cudaSuccess) return W4A4_ERR_CUDA;

@@ -332,7 +332,8 @@ int w4a4_gemm_rope(const uint8_t* Xq, const uint8_t* Xsf, const float* t_x, cons
  *   next_sf     out  SF atoms of the [M, next_K] activation (nvfp4_sf_bytes(M,
  *                    next_K) bytes); the scale bytes of those columns for rows
  *                    < M are written (pad rows are left as they are)
- *   next_K, next_col  next_K % 64 == 0, next_col % 64 == 0, next_col + n_out <= next_K
+ *   next_K, next_col  next_K % 64 == 0, next_K <= W4A4_MAX_K, next_col % 64 == 0,
+ *                    next_col + n_out <= next_K
  *   next_amax   as in w4a4_gemm_next_amax (over F), or NULL
  *   Y / H       as in w4a4_gemm / w4a4_gemm_swiglu; may be NULL to skip
  *               storing the bf16 values (Y must be given when n_plain is
