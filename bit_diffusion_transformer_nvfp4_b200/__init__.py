@@ -26,7 +26,7 @@ __all__ = [
     "nvfp4_quantize_act_noalloc", "nvfp4_quantize_act_with_amax", "w4a4_gemm_next_amax", "w4a4_gemm_swiglu",
     "gemm_swiglu", "w4a4_gemm_quantize_next", "gemm_quantize_next", "w4a4_gemm_rope", "gemm_rope",
     "fp8_quant_workspace_bytes", "fp8_quantize", "attention_fp8", "Fp8Tensor", "quantize_fp8", "attention",
-    "w4a4_fp4_mma_rate", "w4a4_last_error",
+    "w4a4_fp4_mma_rate", "w4a4_last_error", "MAX_K",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +34,7 @@ LIB_PATH = os.path.join(HERE, "libw4a4.so")
 
 EPI_NONE, EPI_GELU_TANH = 0, 1
 SRC_BF16, SRC_F32 = 0, 1
+MAX_K = 1 << 20  # W4A4_MAX_K: the widest K (activation or weight columns) the entry points accept
 
 _c = ctypes
 _P = _c.c_void_p

@@ -90,9 +90,12 @@ def test_k_and_fp8_column_bounds(so):
     """K up to 2^20 (the widest row the tensor-amax pass covers with its 1024
     partial maxima of 256 segments) and FP8 columns up to 2^21 are accepted;
     one step past either bound is a size error before any launch."""
+    import bit_diffusion_transformer_nvfp4_b200 as w
     P = 1 << 20
     big = 1 << 30
     kmax = 1 << 20
+    hdr = open(HEADER).read()
+    assert re.search(r"#define W4A4_MAX_K \(\(int64_t\)1 << 20\)", hdr) and w.MAX_K == kmax
     assert so.nvfp4_quant_workspace_bytes(128, kmax, 32) > 0
     assert so.nvfp4_quant_workspace_bytes(128, kmax + 64, 32) == 0
     assert so.w4a4_workspace_bytes(128, 256, kmax, 32) > 0
