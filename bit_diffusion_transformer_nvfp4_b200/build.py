@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libw4a4.so")
 SOURCES = ["w4a4_api.cu"]
-DEPS = ["w4a4_api.cu", "attention.cuh", "gemm.cuh", "gemm2.cuh", "quant.cuh", "sm100.cuh"]
+DEPS = ["w4a4_api.cu", "attention.cuh", "gemm.cuh", "gemm2.cuh", "mma_rate.cuh", "quant.cuh", "sm100.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
